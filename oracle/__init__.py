@@ -1,0 +1,3 @@
+"""CPU fp64 oracle (test infrastructure only; never imported by the library)."""
+from .attn import (allowed_mask, attn_probs, attn_fwd, attn_rows, attn_bwd, attn_decode,
+                   merge_partials, fwd_flops, allowed_pairs, score_matrix_elements)
