@@ -1,0 +1,392 @@
+"""Benchmark of the exact tiled attention kernels on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+
+Headline (one JSON line on rank 0): causal bf16 prefill forward on
+B=4, Hq=Hkv=16, L=2048, D=128 (Q x4 on heads 0-7, seed 1), in TFLOP/s with the
+causal (query, key) pairs counted once.  A step is one fa_fwd call over the
+whole batch, inputs resident in HBM, L2 flushed before every timed step.  The
+same line carries, under "sections", the other workloads measured in the same
+run (long-context GQA prefill, training forward+backward, split-KV decode).
+
+Multi-GPU: replicas only (every rank runs the same workload on its own copy;
+no collective on the data path); value = all ranks' FLOPs / max-over-ranks time.
+
+--impl reference times the CPU fp64 oracle on a bounded sample of the same
+workload (rank 0 only), as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_tiled_attention_46_b200 import inputs as synth  # noqa: E402
+
+METRIC = "attn fwd/bwd TFLOP/s & % BF16 tensor peak; decode KV-read GB/s & % of HBM"
+HEADLINE = "causal_prefill"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def allowed_pairs(Lq, Lk, causal):
+    if not causal:
+        return Lq * Lk
+    off = Lk - Lq
+    i = np.arange(Lq, dtype=np.int64)
+    return int(np.clip(i + off + 1, 0, Lk).sum())
+
+
+def fwd_flops(w):
+    return 4.0 * w.B * w.Hq * w.D * allowed_pairs(w.Lq, w.Lk, w.causal)
+
+
+def fwd_bytes(w):
+    # Q, K, V read once, O written once (bf16), LSE written (fp32)
+    return 2.0 * (2 * w.B * w.Lq * w.Hq * w.D + 2 * w.B * w.Lk * w.Hkv * w.D) + 4.0 * w.B * w.Hq * w.Lq
+
+
+# ----------------------------------------------------------------- clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        busy = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------- our arm -----
+def l2_flusher(dev):
+    buf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        buf.fill_(1.0)
+    return flush
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s, e in evs:
+        flush()
+        s.record(stream)
+        fn()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+def section_fwd(fa, name, steps, warmup, flush, stream, peaks, dev):
+    w = synth.WORKLOADS[name]
+    x = synth.workload_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+    ms = time_steps(lambda: fa.fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse), steps, warmup, flush,
+                    stream)
+    t = statistics.mean(ms) * 1e-3
+    tf = fwd_flops(w) / t / 1e12
+    return {"workload": name, "kernel": "fwd_kernel", "ms": t * 1e3, "tflops": tf,
+            "frac_bf16_peak": tf / peaks["bf16_tflops"], "launches": steps}
+
+
+def section_train(fa, steps, warmup, flush, stream, peaks, dev):
+    w = synth.WORKLOADS["train_fwd_bwd"]
+    x = synth.workload_inputs(w)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = fa.fwd(q, k, v, scale=w.scale, causal=w.causal)
+    ws = torch.empty(fa.bwd_workspace_size(w.B, w.Hq, w.Lq, w.D), dtype=torch.uint8, device=dev)
+    try:
+        fa.bwd(q, k, v, o, do, lse, scale=w.scale, causal=w.causal, workspace=ws)
+    except fa.FaError as e:
+        return {"workload": "train_fwd_bwd", "unavailable": str(e)}
+
+    def step():
+        fa.fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+        fa.bwd(q, k, v, o, do, lse, scale=w.scale, causal=w.causal, workspace=ws)
+    ms = time_steps(step, steps, warmup, flush, stream)
+    t = statistics.mean(ms) * 1e-3
+    ms_b = time_steps(lambda: fa.bwd(q, k, v, o, do, lse, scale=w.scale, causal=w.causal, workspace=ws),
+                      steps, warmup, flush, stream)
+    tb = statistics.mean(ms_b) * 1e-3
+    ff = fwd_flops(w)
+    return {"workload": "train_fwd_bwd", "ms_fwd_bwd": t * 1e3, "tflops_fwd_bwd": 3.5 * ff / t / 1e12,
+            "ms_bwd": tb * 1e3, "tflops_bwd": 2.5 * ff / tb / 1e12,
+            "frac_bf16_peak_fwd_bwd": 3.5 * ff / t / 1e12 / peaks["bf16_tflops"]}
+
+
+def section_decode(fa, steps, warmup, flush, stream, peaks, dev):
+    w = synth.WORKLOADS["splitkv_decode"]
+    x = synth.decode_inputs(w.B, w.Hq, w.Hkv, w.Lk, w.D, w.seed, w.len_lo, w.len_hi, device=dev)
+    q, kc, vc, sl = x["q"].to(dev), x["k_cache"], x["v_cache"], x["seqlens"].to(dev)
+    ws = torch.empty(fa.decode_workspace_size(w.B, w.Hq, w.Lk, w.D), dtype=torch.uint8, device=dev)
+    o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ms = time_steps(lambda: fa.decode(q, kc, vc, sl, scale=w.scale, workspace=ws, out=o, lse=lse), steps, warmup,
+                    flush, stream)
+    t = statistics.mean(ms) * 1e-3
+    kv_bytes = float(x["seqlens"].to(torch.int64).sum()) * w.Hkv * w.D * 2 * 2
+    gbs = kv_bytes / t / 1e9
+    return {"workload": "splitkv_decode", "kernel": "decode_split_kernel+decode_combine_kernel", "ms": t * 1e3,
+            "kv_bytes": kv_bytes, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "launches": 2 * steps}
+
+
+def run_ours(args):
+    import exact_tiled_attention_46_b200 as fa
+    from exact_tiled_attention_46_b200 import build
+    build.build()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush = l2_flusher(dev)
+    w = synth.WORKLOADS[HEADLINE]
+    x = synth.workload_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+
+    def step():
+        fa.fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+    # timed region: barrier + sync on both sides, per-step CUDA events on the launching stream
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
+    region0.record(stream)
+    for s, e in evs:
+        flush()
+        s.record(stream)
+        step()
+        e.record(stream)
+    region1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ck = clocks.stop() if rank == 0 else None
+    kernel_ms = sum(s.elapsed_time(e) for s, e in evs)
+    t_local = torch.tensor([kernel_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    kernel_ms = float(t_local.item())
+    ms_step = kernel_ms / args.steps
+    flops = fwd_flops(w)
+    value = flops * world * args.steps / (kernel_ms * 1e-3) / 1e12
+    tf_rank = flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device -> fwd -> host
+    hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        fa.fwd(dq, dk, dv, scale=w.scale, causal=w.causal, out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+    e2e_ms = statistics.mean(time_steps(e2e_step, max(3, args.steps // 4), 2, flush, stream))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    e2e_val = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    sections = {}
+    if not args.quick:
+        sec_steps = max(3, min(args.steps, 20))
+        sections["long_gqa_prefill"] = section_fwd(fa, "long_gqa_prefill", sec_steps, 3, flush, stream, peaks, dev)
+        sections["train_fwd_bwd"] = section_train(fa, sec_steps, 3, flush, stream, peaks, dev)
+        sections["splitkv_decode"] = section_decode(fa, sec_steps, 3, flush, stream, peaks, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(budget_s=args.cpu_budget)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16 RNE)",
+        "config": {"workload": "causal_prefill B4 Hq16 Hkv16 L2048 D128 causal, Q x4 on heads 0-7",
+                   "global_batch": w.B * world, "seq_len": w.Lq, "heads": w.Hq, "head_dim": w.D,
+                   "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) before every timed step",
+                   "flops_per_step": flops, "flop_count": "4*B*H*D*allowed_pairs, causal pairs counted once"},
+        "roofline": {"bound": "tensor", "achieved": tf_rank, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tf_rank / peak, "traffic": None, "peak_source": f"{peak_src} bf16 burst",
+                     "algorithmic_bytes": fwd_bytes(w)},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": ck,
+        "sections": sections,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------- oracle timing ---
+def oracle_sample(w, n_heads, rng_seed=0):
+    """The oracle on the first n_heads (batch, head) slices of the workload."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    x = synth.workload_inputs(w)
+    xf = {n: synth.as_f64(x[n]) for n in ("q", "k", "v")}
+    G = w.Hq // w.Hkv
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hq)][:n_heads]
+    t0 = time.perf_counter()
+    for b, h in pairs:
+        oracle.attn_fwd(xf["q"][b:b + 1, :, h:h + 1], xf["k"][b:b + 1, :, h // G:h // G + 1],
+                        xf["v"][b:b + 1, :, h // G:h // G + 1], w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.D * allowed_pairs(w.Lq, w.Lk, w.causal) * len(pairs)
+    return flops, dt
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(budget_s=15.0):
+    w = synth.WORKLOADS[HEADLINE]
+    f1, t1 = oracle_sample(w, 1)
+    n = max(1, min(w.B * w.Hq, int(budget_s / max(t1, 1e-3))))
+    f, t = oracle_sample(w, n)
+    return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{n} of {w.B * w.Hq} (batch, head) slices of causal_prefill, NumPy fp64, {t:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[HEADLINE]
+    oracle_sample(w, 1)   # warm imports / BLAS threads
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_sample(w, 1)
+    per = []
+    flops_total, t_total = 0.0, 0.0
+    for _ in range(args.steps):
+        f, t = oracle_sample(w, 2)
+        per.append(t)
+        flops_total += f
+        t_total += t
+    value = flops_total / t_total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), bf16 RNE)",
+        "config": {"workload": "causal_prefill B4 Hq16 Hkv16 L2048 D128 causal, Q x4 on heads 0-7",
+                   "sample_per_step": "2 (batch, head) slices"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": "2 (batch, head) slices of causal_prefill per step, NumPy fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline only, no extra sections")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

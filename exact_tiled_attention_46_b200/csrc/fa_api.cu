@@ -1,0 +1,289 @@
+// Host side of the C ABI declared in include/fa.h: argument checks, tensor-map
+// encoding, kernel selection and launches.  Nothing here allocates device
+// memory or synchronises (except fa_device_status, which says so).
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "sm100.cuh"
+#include "fa_fwd.cuh"
+#include "fa_decode.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr int kDecodeChunk = 1024;
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+// ---------------------------------------------------------- tensor maps ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 4-D map over a [B, L, H, D] bf16 tensor: dims (D, H, L, B), box (box_d, 1, box_rows, 1).
+bool map_bshd(CUtensorMap* m, const void* base, int B, int L, int H, int D, int box_d, int box_rows, bool sw128) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(L), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2, cuuint64_t(L) * H * D * 2};
+  cuuint32_t box[4] = {cuuint32_t(box_d), 1, cuuint32_t(box_rows), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- helpers -----
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+bool fits_int(long long x) { return x >= 0 && x <= INT_MAX; }
+
+// Sets the dynamic shared-memory limit of `func` once per device.
+template <typename F>
+bool ensure_smem_attr(F* func, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done_mask.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+fa_status launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+__global__ void fill_empty_rows_kernel(void* o, float* lse, size_t n_o, size_t n_lse, int o_fp32) {
+  const size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x;
+  const size_t stride = size_t(gridDim.x) * blockDim.x;
+  for (size_t k = i; k < n_o; k += stride) {
+    if (o_fp32) static_cast<float*>(o)[k] = 0.f;
+    else static_cast<uint16_t*>(o)[k] = 0;
+  }
+  if (lse != nullptr)
+    for (size_t k = i; k < n_lse; k += stride) lse[k] = -INFINITY;
+}
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) { fa::mbar_init(&bar, 1); fa::fence_mbar_init(); }
+  __syncthreads();
+  fa::mbar_wait(&bar, 0, limit_ns, 0x9001);   // no thread ever arrives
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
+                     long long grid, cudaStream_t st) {
+  static std::atomic<uint64_t> attr_done{0};
+  constexpr int smem = fa::FwdCfg<D>::SMEM_BYTES;
+  if (!ensure_smem_attr(fa::fwd_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
+  fa::fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), fa::FwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+template <int D, int GP>
+fa_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p, dim3 grid,
+                        cudaStream_t st) {
+  static std::atomic<uint64_t> attr_done{0};
+  using C = fa::DecCfg<D, GP>;
+  if (!ensure_smem_attr(fa::decode_split_kernel<D, GP>, C::SMEM_BYTES, attr_done)) return FA_ERR_CUDA;
+  fa::decode_split_kernel<D, GP><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mk, mv, p);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_abi_version(void) { return kAbiVersion; }
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_CUDA: return "CUDA call failed";
+    case FA_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+void fa_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns > 0 ? ns : 1); }
+
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                    int Lq, int Lk, int D, float scale, int causal, int o_dtype, fa_stream_t stream) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  // empty tensors may come with null pointers: q/o only matter when Lq > 0, k/v when Lk > 0
+  if (Lq > 0 && (!q || !o)) return FA_ERR_INVALID_ARG;
+  if (Lq > 0 && Lk > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const long long pairs = (static_cast<long long>(Lq) + 255) / 256;
+  const long long grid = pairs * B * Hq;
+  if (!fits_int(grid) || !fits_int(static_cast<long long>(B) * Hq)) return FA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Lq == 0) return FA_OK;
+  if (Lk == 0) {
+    const size_t n_o = size_t(B) * Lq * Hq * D, n_l = size_t(B) * Hq * Lq;
+    fill_empty_rows_kernel<<<296, 256, 0, st>>>(o, lse, n_o, n_l, o_dtype == FA_FP32);
+    return launch_status();
+  }
+  CUtensorMap mq, mk, mv;
+  if (!map_bshd(&mq, q, B, Lq, Hq, D, 64, 128, true) || !map_bshd(&mk, k, B, Lk, Hkv, D, 64, 128, true) ||
+      !map_bshd(&mv, v, B, Lk, Hkv, D, 64, 128, true))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = o; p.lse = lse; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk;
+  p.num_pairs = static_cast<int>(pairs);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_fp32 = (o_dtype == FA_FP32);
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  if (D == 128) return causal ? launch_fwd<128, true>(mq, mk, mv, p, grid, st) : launch_fwd<128, false>(mq, mk, mv, p, grid, st);
+  return causal ? launch_fwd<64, true>(mq, mk, mv, p, grid, st) : launch_fwd<64, false>(mq, mk, mv, p, grid, st);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                 int Lk, int D, float scale, int causal, fa_stream_t stream) {
+  return fa_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, FA_BF16, stream);
+}
+
+int fa_decode_chunk(void) { return kDecodeChunk; }
+
+size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int D) {
+  if (B <= 0 || Hq <= 0 || Lmax < 0 || D <= 0) return 0;
+  const size_t ms = std::max<size_t>(1, (size_t(Lmax) + kDecodeChunk - 1) / kDecodeChunk);
+  return align_up(size_t(B) * Hq * ms * D * 4, 256) + align_up(size_t(B) * Hq * ms * 4, 256);
+}
+
+fa_status fa_decode_combine(const float* o_part, const float* lse_part, const int* num_splits, void* o, float* lse,
+                            int B, int Hq, int D, int max_splits, int o_dtype, fa_stream_t stream) {
+  if (!o_part || !lse_part || !o) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || D <= 0 || D > 4096 || max_splits <= 0) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (!fits_int(static_cast<long long>(B) * Hq)) return FA_ERR_UNSUPPORTED;
+  fa::CombineParams c;
+  c.o_part = o_part; c.lse_part = lse_part; c.counts = num_splits; c.o = o; c.lse = lse;
+  c.B = B; c.Hq = Hq; c.D = D; c.max_splits = max_splits; c.chunk = 0; c.o_fp32 = (o_dtype == FA_FP32);
+  fa::decode_combine_kernel<<<B * Hq, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c);
+  return launch_status();
+}
+
+fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, void* o,
+                            float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, int o_dtype,
+                            void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !seqlens || !o || !workspace) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned256(workspace))
+    return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) != 0 || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  const int GP = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+  const int max_splits = (Lmax + kDecodeChunk - 1) / kDecodeChunk;
+  if (max_splits > 65535 || Hkv * (G / GP) > 65535 || B > 65535) return FA_ERR_UNSUPPORTED;
+  if (workspace_bytes < fa_decode_workspace_size(B, Hq, Lmax, D)) return FA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap mk, mv;
+  if (!map_bshd(&mk, k_cache, B, Lmax, Hkv, D, D, fa::DecCfg<128, 4>::T, false) ||
+      !map_bshd(&mv, v_cache, B, Lmax, Hkv, D, D, fa::DecCfg<128, 4>::T, false))
+    return FA_ERR_CUDA;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             align_up(size_t(B) * Hq * max_splits * D * 4, 256));
+  fa::DecParams p;
+  p.seqlens = seqlens; p.q = static_cast<const uint16_t*>(q); p.o_part = o_part; p.lse_part = lse_part;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = Lmax; p.max_splits = max_splits; p.chunk = kDecodeChunk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const dim3 grid(max_splits, Hkv * (G / GP), B);
+  fa_status s;
+  if (D == 128) s = GP == 4 ? launch_decode<128, 4>(mk, mv, p, grid, st)
+                  : GP == 2 ? launch_decode<128, 2>(mk, mv, p, grid, st) : launch_decode<128, 1>(mk, mv, p, grid, st);
+  else s = GP == 4 ? launch_decode<64, 4>(mk, mv, p, grid, st)
+         : GP == 2 ? launch_decode<64, 2>(mk, mv, p, grid, st) : launch_decode<64, 1>(mk, mv, p, grid, st);
+  if (s != FA_OK) return s;
+  fa::CombineParams c;
+  c.o_part = o_part; c.lse_part = lse_part; c.counts = seqlens; c.o = o; c.lse = lse;
+  c.B = B; c.Hq = Hq; c.D = D; c.max_splits = max_splits; c.chunk = kDecodeChunk; c.o_fp32 = (o_dtype == FA_FP32);
+  fa::decode_combine_kernel<<<B * Hq, 128, 0, st>>>(c);
+  return launch_status();
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D) {
+  if (B <= 0 || Hq <= 0 || Lq < 0 || D <= 0) return 0;
+  const size_t lq_pad = align_up(size_t(Lq), 128);
+  return align_up(size_t(B) * Lq * Hq * D * 4, 256) + align_up(size_t(B) * Hq * lq_pad * 4, 256);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int causal,
+                 int grad_dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (grad_dtype != FA_BF16 && grad_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned256(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (workspace_bytes < fa_bwd_workspace_size(B, Hq, Lq, D)) return FA_ERR_INVALID_ARG;
+  return fa::bwd_dispatch(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, Lq, Lk, D, scale, causal,
+                          grad_dtype == FA_FP32, workspace, reinterpret_cast<cudaStream_t>(stream),
+                          g_wait_limit_ns.load());
+}
+
+fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t s = 0, w = 0;
+  if (cudaMemcpyFromSymbolAsync(&s, fa::g_fa_dev_status, 4, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyFromSymbolAsync(&w, fa::g_fa_dev_where, 4, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (code) *code = (s == fa::FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : FA_OK;
+  if (where) *where = static_cast<int>(w);
+  if (reset) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbolAsync(fa::g_fa_dev_status, &zero, 4, 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(fa::g_fa_dev_where, &zero, 4, 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t stream) {
+  if (wait_ns == 0 || wait_ns > 10000000000ull) return FA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(wait_ns);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,316 @@
+// Prefill forward: exact softmax(Q K^T * scale) V, tile by tile with an online
+// softmax ("FlashAttention Explained: How AI Models Process Attention Faster
+// and Use Less Memory", sections "1. Tiling", "3. Online Softmax" and "Fused
+// Computation"; "Flash Attention Explained: Same Maths, Far Less Memory",
+// section "The idea: never materialise the matrix").  The score matrix lives
+// only in tensor memory; HBM sees Q, K, V once per CTA and O/LSE once.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and walks the key
+// tiles of its kv head:
+//   warp 8      TMA producer: Q tiles once, then K_j, V_j into a slot ring
+//   warp 9      MMA issuer:   S_t = Q_t K_j^T into TMEM, O_t += P_t V_j
+//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one
+//               thread per query row; causal / ragged mask; running max m and
+//               running sum l in log2 units; P (bf16) written over S in TMEM;
+//               O rescaled in TMEM only when the max grows by more than TAU;
+//               epilogue O / l and LSE.
+//   warp 10     allocates / frees the 512 TMEM columns.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
+#pragma once
+#include "sm100.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  void* o;                 // [B, Lq, Hq, D] bf16 or fp32
+  float* lse;              // [B, Hq, Lq] or nullptr
+  int B, Hq, Hkv, Lq, Lk;
+  int num_pairs;           // ceil(Lq / 256)
+  float scale_log2;        // scale * log2(e)
+  int o_fp32;
+  uint64_t wait_limit_ns;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;       // one 128-row bf16 tile
+  static constexpr int NS = (D == 128) ? 4 : 8;        // K/V slots
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
+  static constexpr int NBARS = 1 + 2 * NS + 2 + 2 + 2 + 1;
+  static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
+  static constexpr int THREADS = 384;
+};
+
+// rescale O only when the running max grows by more than 2^8 (log2 units);
+// otherwise the stale max stays the reference and P <= 2^8.
+constexpr float FWD_TAU = 8.0f;
+
+enum : uint32_t {
+  W_FWD_Q = 0x101, W_FWD_KV_EMPTY = 0x102, W_FWD_KV_FULL = 0x103, W_FWD_P = 0x104,
+  W_FWD_S = 0x105, W_FWD_O = 0x106, W_FWD_DONE = 0x107, W_FWD_DRAIN = 0x108
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::NS;
+  constexpr int KB = D / 64;                       // 64-column (128-byte) blocks per row
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* bar_q = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit_ns;
+
+  // heaviest query-tile pairs first (causal work grows with the pair index)
+  const int bh_count = p.B * p.Hq;
+  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x / bh_count);
+  const int bh = static_cast<int>(blockIdx.x % bh_count);
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int hkv = h / (p.Hq / p.Hkv);
+  const int q0 = pair * 256;
+  const int off = p.Lk - p.Lq;                     // bottom-right causal alignment
+  const int nk_all = (p.Lk + 127) >> 7;
+
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = q0 + t * 128;
+    if (r0 >= p.Lq) {
+      n_t[t] = 0;
+    } else if (!CAUSAL) {
+      n_t[t] = nk_all;
+    } else {
+      const int lim_keys = min(r0 + 127, p.Lq - 1) + off + 1;   // keys < lim_keys for the last row
+      n_t[t] = lim_keys <= 0 ? 0 : min(nk_all, (lim_keys + 127) >> 7);
+    }
+  }
+  const int n = max(n_t[0], n_t[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    for (int t = 0; t < 2; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_full[t], 1); }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 10) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  if (warp == 8 && lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0 && n > 0) {
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+      for (int t = 0; t < 2; ++t)
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_4d(smem + C::Q_OFF + t * C::TILE_BYTES + kb * 16384, &tm_q, bar_q, kb * 64, h, q0 + t * 128, b);
+      int issued = 0;
+      for (int it = 0; it < 2 * n; ++it) {
+        const int slot = it % NS;
+        if (it >= NS && !mbar_wait(&kv_empty[slot], ((it / NS) + 1) & 1, lim, W_FWD_KV_EMPTY)) break;
+        mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
+        const CUtensorMap* m = (it & 1) ? &tm_v : &tm_k;
+        uint8_t* dst = smem + C::KV_OFF + slot * C::TILE_BYTES;
+        for (int kb = 0; kb < KB; ++kb) tma_load_4d(dst + kb * 16384, m, &kv_full[slot], kb * 64, hkv, (it >> 1) * 128, b);
+        issued = it + 1;
+      }
+      // the CTA may not exit with copies in flight: wait for the last loads
+      mbar_wait(bar_q, 0, lim, W_FWD_DRAIN);
+      for (int it = max(0, issued - NS); it < issued; ++it)
+        mbar_wait(&kv_full[it % NS], (it / NS) & 1, lim, W_FWD_DRAIN);
+    }
+  } else if (warp == 9) {
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_base = smem_u32(smem + C::Q_OFF);
+      const uint32_t kv_base = smem_u32(smem + C::KV_OFF);
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = q_base + t * C::TILE_BYTES, ka = kv_base + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + t * 128, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), IDESC_S, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t va = kv_base + slot * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), IDESC_O,
+                  (acc || kk > 0) ? 1u : 0u);
+      };
+      auto wait_item = [&](int it) { return mbar_wait(&kv_full[it % NS], (it / NS) & 1, lim, W_FWD_KV_FULL); };
+
+      bool ok = mbar_wait(bar_q, 0, lim, W_FWD_Q) && wait_item(0);
+      tc_fence_after();
+      if (ok) {
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) { issue_s(t, 0); umma_commit(&s_full[t]); }
+        umma_commit(&kv_empty[0]);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int it_v = 2 * j + 1, it_k = 2 * j + 2;
+        if (!(ok = wait_item(it_v))) break;
+        tc_fence_after();
+        bool k_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_t[t]) continue;
+          if (!(ok = mbar_wait(&p_full[t], j & 1, lim, W_FWD_P))) break;
+          tc_fence_after();
+          issue_pv(t, it_v % NS, j > 0);
+          if (j + 1 < n_t[t]) {
+            if (!k_ready) {
+              if (!(ok = wait_item(it_k))) break;
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_s(t, it_k % NS);
+            umma_commit(&s_full[t]);
+          } else {
+            umma_commit(&o_full[t]);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[it_v % NS]);
+        if (k_ready) umma_commit(&kv_empty[it_k % NS]);
+      }
+      // nothing may be in flight on the tensor pipe when the CTA tears down
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, lim, W_FWD_DONE);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------- softmax --
+    const int t = warp >> 2;
+    const int wq = warp & 3;                       // TMEM lane quadrant of this warp
+    const int row = q0 + t * 128 + wq * 32 + lane; // global query row of this thread
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem + lane_bits + t * 128;
+    const uint32_t t_o = tmem + lane_bits + 256 + t * D;
+    const int nt = n_t[t];
+    const float sl2 = p.scale_log2;
+    const int row_tile0 = q0 + t * 128;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+
+    for (int j = 0; j < nt; ++j) {
+      if (!(ok = mbar_wait_warp(&s_full[t], j & 1, lim, W_FWD_S))) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld_32x32b_x128(t_s, sr);
+      float* s = reinterpret_cast<float*>(sr);
+      const int kbase = j * 128;
+      const bool need_mask = (kbase + 128 > p.Lk) || (CAUSAL && kbase + 127 > row_tile0 + off);
+      if (need_mask) {
+        int lim_c = p.Lk - kbase;
+        if (CAUSAL) lim_c = min(lim_c, row + off + 1 - kbase);
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = (c < lim_c) ? s[c] : -INFINITY;
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]); mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const bool resc = m_tile > m_used + FWD_TAU;   // false while both are -inf
+      float alpha = 1.f;
+      if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; m_used = m_tile; }
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(t_o + c0, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st_32x32b_x32(t_o + c0, ov);
+        }
+      }
+      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = half * 64 + 2 * i;
+          const float p0 = ex2_approx(fmaf(s[c], sl2, -msub));
+          const float p1 = ex2_approx(fmaf(s[c + 1], sl2, -msub));
+          ls0 += p0; ls1 += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_32x32b_x32(t_s + half * 32, pk);   // P over the first 64 columns of S
+      }
+      l += ls0 + ls1;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // ------------------------------------------------------------ epilogue --
+    const bool have_o = ok && nt > 0 && mbar_wait_warp(&o_full[t], 0, lim, W_FWD_O);
+    if (have_o) tc_fence_after();
+    const bool has = l > 0.f;
+    const float inv_l = has ? 1.f / l : 0.f;
+    const bool in_range = row < p.Lq;
+    if (in_range && p.lse != nullptr)
+      p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_used + log2f(l)) * LN2 : -INFINITY;
+    const size_t orow = (static_cast<size_t>(b) * p.Lq + row) * p.Hq + h;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t ov[32];
+      if (have_o) {
+        tmem_ld_32x32b_x32(t_o + c0, ov);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0u;
+      }
+      if (!in_range) continue;
+      if (p.o_fp32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
+                               __uint_as_float(ov[4 * i + 2]) * inv_l, __uint_as_float(ov[4 * i + 3]) * inv_l);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]) * inv_l, __uint_as_float(ov[8 * i + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]) * inv_l, __uint_as_float(ov[8 * i + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]) * inv_l, __uint_as_float(ov[8 * i + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]) * inv_l, __uint_as_float(ov[8 * i + 7]) * inv_l);
+          dst[i] = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 10) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

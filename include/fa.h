@@ -1,0 +1,151 @@
+/*
+ * fa.h: C ABI of the exact tiled attention library (sm_100a, B200).
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(Q K^T * scale) V
+ * ("FlashAttention Explained: How AI Models Process Attention Faster and Use
+ * Less Memory", section "Understanding Attention in Transformer Models") tile
+ * by tile with an online softmax (same page, "3. Online Softmax"; "Flash
+ * Attention Explained: Same Maths, Far Less Memory", "The idea: never
+ * materialise the matrix"), so that the score matrix is never written to
+ * device memory.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers to contiguous row-major memory
+ *     owned by the caller.  bf16 tensors must be 16-byte aligned.
+ *   - Layouts: q, o, dO, dq        [B, Lq, Hq, D]
+ *              k, v, dk, dv        [B, Lk, Hkv, D]
+ *              lse, delta          [B, Hq, Lq]     (fp32, natural log)
+ *              decode q, o         [B, Hq, D];  cache [B, Lmax, Hkv, D]
+ *   - D is 64 or 128; Hq must be a multiple of Hkv; query head h reads kv
+ *     head h / (Hq / Hkv) (grouped-query attention, "Flash Attention
+ *     Explained: Same Maths, Far Less Memory", "What it does not solve").
+ *   - causal != 0 allows key j for query i when j <= i + (Lk - Lq)
+ *     (bottom-right alignment).  A query with no allowed key gets O = 0 and
+ *     LSE = -inf.
+ *   - scale must be finite and > 0 (1/sqrt(D) is the pages' choice).
+ *   - stream is a cudaStream_t (may be 0).  Every call only enqueues work: it
+ *     never synchronises and never allocates.  Arguments are checked before
+ *     anything is launched; a bad argument returns FA_ERR_INVALID_ARG or
+ *     FA_ERR_UNSUPPORTED and launches nothing.  A failed launch returns
+ *     FA_ERR_CUDA.  Device-side faults surface at the caller's next
+ *     synchronisation; a kernel wait that runs out of time is reported by
+ *     fa_device_status() (the kernel then returns instead of hanging).
+ *   - The library keeps two device words of state (the device status) and a
+ *     per-device record of kernel attributes set; calls are thread-safe.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, workspace too small */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented here (e.g. D not in {64,128}) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+  FA_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fa_device_status) */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP32 = 1 } fa_dtype;
+
+/* Version of this ABI (incremented on any signature change). */
+int fa_abi_version(void);
+
+/* Static text for a status code; never NULL. */
+const char* fa_status_string(int status);
+
+/*
+ * Prefill forward.  Reads q, k, v (bf16); writes o (bf16) and, when lse is
+ * not NULL, lse (fp32, ln of the softmax denominator including the max).
+ * Lq == 0 is a no-op; Lk == 0 writes O = 0 and LSE = -inf.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int causal,
+                 fa_stream_t stream);
+
+/* As fa_fwd, with the output dtype of o chosen (FA_BF16 or FA_FP32). */
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int causal,
+                    int o_dtype, fa_stream_t stream);
+
+/*
+ * Backward ("FlashAttention Explained ...", section "More Efficient
+ * Backpropagation"; "How FlashAttention Speeds Up LLM Attention", "Recompute
+ * probabilities for training"): probabilities are recomputed per tile from q,
+ * k and the saved lse instead of being stored.  Reads q, k, v, o, dO (bf16)
+ * and lse (fp32, as written by fa_fwd); writes dq [B,Lq,Hq,D], dk and dv
+ * [B,Lk,Hkv,D] in grad_dtype (FA_BF16 or FA_FP32).  dk/dv of a kv head are the
+ * sums over its Hq/Hkv query heads.  workspace is caller-owned device memory
+ * of at least fa_bwd_workspace_size() bytes (256-byte aligned); its contents
+ * on entry do not matter.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D);
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int causal,
+                 int grad_dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Split-KV decode ("Flash Attention Explained: Same Maths, Far Less Memory",
+ * "Where you actually feel it"): one query per (sequence, head) against the
+ * first seqlens[b] rows of a contiguous cache.  q [B,Hq,D] bf16; k_cache,
+ * v_cache [B,Lmax,Hkv,D] bf16; seqlens int32 [B] on the device (values are
+ * clamped to [0, Lmax]; rows at or past seqlens[b] are never read into the
+ * result); o [B,Hq,D] in o_dtype; lse [B,Hq] fp32 or NULL.  The cache is cut
+ * into chunks of fa_decode_chunk() keys; each chunk's partial result goes to
+ * the workspace (>= fa_decode_workspace_size() bytes, 256-byte aligned) and a
+ * second kernel combines them.  Two launches on `stream`.
+ */
+int fa_decode_chunk(void);
+size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int D);
+fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                            const int* seqlens, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                            int o_dtype, void* workspace, size_t workspace_bytes,
+                            fa_stream_t stream);
+
+/*
+ * Combine partial results over disjoint key sets (the merge step of split-KV
+ * decode; "How FlashAttention Speeds Up LLM Attention": partial results kept
+ * on the same numerical scale).  o_part [B,Hq,max_splits,D] fp32 holds
+ * normalised partial outputs, lse_part [B,Hq,max_splits] fp32 their natural
+ * log-sum-exps (-inf for an empty part).  num_splits [B] int32 on the device
+ * gives how many leading parts of sequence b are valid (NULL: all
+ * max_splits).  Writes o [B,Hq,D] in o_dtype and lse [B,Hq] (or NULL):
+ * lse = ln sum_s exp(lse_s), o = sum_s exp(lse_s - lse) o_s.
+ */
+fa_status fa_decode_combine(const float* o_part, const float* lse_part, const int* num_splits,
+                            void* o, float* lse, int B, int Hq, int D, int max_splits,
+                            int o_dtype, fa_stream_t stream);
+
+/*
+ * Device status of the current device: *code receives 0 (ok) or FA_ERR_TIMEOUT
+ * when some kernel's bounded wait ran out since the last reset, *where a code
+ * naming the wait.  Synchronises `stream`.  reset != 0 clears the status.
+ */
+fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream);
+
+/*
+ * Upper bound, in nanoseconds, on any single wait inside a kernel (default
+ * 2e9).  Process-wide; affects launches made after the call.
+ */
+void fa_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Self-test of the bounded wait: launches one block that waits on a barrier
+ * nothing ever completes, with a limit of wait_ns nanoseconds; the kernel
+ * records FA_ERR_TIMEOUT in the device status and returns.
+ */
+fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FA_H_ */

@@ -1,0 +1,55 @@
+"""Shared helpers of the GPU parity tests (tolerances, device tensors)."""
+import numpy as np
+import pytest
+import torch
+
+# Tolerances for floating point outputs: max-abs 1e-2 and mean-abs 1e-3 on O and
+# the gradients, 1e-3 absolute on LSE.  For bf16 outputs the tolerance is applied
+# on top of the output format's own rounding: half the bf16 spacing at the exact
+# value (2^-9 relative), since a perfectly rounded bf16 value of magnitude >= 4
+# already differs from the exact one by up to 2^-6.
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+LSE_ABS = 1e-3
+
+
+def bf16_half_spacing(ref):
+    a = np.maximum(np.abs(ref), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 8)
+
+
+def check_close(got, ref, bf16_output, what="output", max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    slack = bf16_half_spacing(ref) if bf16_output else np.zeros_like(ref)
+    worst = np.argmax(err - slack)
+    assert np.all(err <= max_abs + slack), \
+        f"{what}: max err {err.flat[worst]:.3e} at {np.unravel_index(worst, err.shape)} (ref {ref.flat[worst]:.4f})"
+    assert err.mean() <= mean_abs + slack.mean(), f"{what}: mean err {err.mean():.3e}"
+
+
+def check_lse(got, ref, what="lse"):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    inf_ref = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(got), inf_ref), f"{what}: -inf pattern differs"
+    if (~inf_ref).any():
+        err = np.abs(got[~inf_ref] - ref[~inf_ref])
+        assert err.max() <= LSE_ABS, f"{what}: max err {err.max():.3e}"
+
+
+def need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    major, minor = torch.cuda.get_device_capability()
+    if (major, minor) != (10, 0):
+        pytest.skip(f"needs sm_100 (B200), found sm_{major}{minor}")
+    from exact_tiled_attention_46_b200 import build
+    build.build()
+
+
+def f64(t):
+    return t.detach().to("cpu").to(torch.float64).numpy()

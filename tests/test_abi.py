@@ -1,0 +1,112 @@
+"""The C-ABI library loads, exports every symbol include/fa.h declares, and
+rejects bad arguments before it touches the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_tiled_attention_46_b200 as fa
+from exact_tiled_attention_46_b200 import build as fabuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fabuild.build()
+    return fa.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "fa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_abi_version_and_strings(L):
+    assert L.fa_abi_version() == 1
+    for code in range(5):
+        assert L.fa_status_string(code)
+    assert L.fa_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(L):
+    # decode: o_part [B,Hq,S,D] fp32 + lse_part [B,Hq,S] fp32, each 256-byte aligned
+    S = -(-32768 // fa.decode_chunk())
+    assert fa.decode_workspace_size(64, 32, 32768, 128) >= 64 * 32 * S * 129 * 4
+    # backward: fp32 dQ accumulator + per-row Delta
+    assert fa.bwd_workspace_size(8, 16, 4096, 64) >= 8 * 4096 * 16 * 64 * 4 + 8 * 16 * 4096 * 4
+    assert fa.bwd_workspace_size(0, 1, 1, 64) == 0
+
+
+P16 = 4096  # a fake, 16-byte aligned "device" address: never dereferenced on these paths
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, P16, P16, P16, None, 1, 1, 1, 8, 8, 64, 0.1, 0, None), fa.FA_ERR_INVALID_ARG),   # null q
+    ((P16, None, P16, P16, None, 1, 1, 1, 8, 8, 64, 0.1, 0, None), fa.FA_ERR_INVALID_ARG),   # null k
+    ((P16, P16, P16, P16, None, 1, 1, 1, 8, 8, 96, 0.1, 0, None), fa.FA_ERR_UNSUPPORTED),    # D=96
+    ((P16, P16, P16, P16, None, 1, 3, 2, 8, 8, 64, 0.1, 0, None), fa.FA_ERR_INVALID_ARG),    # Hq % Hkv
+    ((P16 + 2, P16, P16, P16, None, 1, 1, 1, 8, 8, 64, 0.1, 0, None), fa.FA_ERR_INVALID_ARG),  # misaligned
+    ((P16, P16, P16, P16, None, 1, 1, 1, 8, 8, 64, -1.0, 0, None), fa.FA_ERR_INVALID_ARG),   # scale <= 0
+    ((P16, P16, P16, P16, None, 1, 1, 1, 8, 8, 64, float("nan"), 0, None), fa.FA_ERR_INVALID_ARG),
+    ((P16, P16, P16, P16, None, 0, 1, 1, 8, 8, 64, 0.1, 0, None), fa.FA_ERR_INVALID_ARG),    # B = 0
+    ((P16, P16, P16, P16, None, 1, 1, 1, -1, 8, 64, 0.1, 0, None), fa.FA_ERR_INVALID_ARG),   # Lq < 0
+])
+def test_fwd_rejects_bad_arguments(L, args, expect):
+    assert L.fa_fwd(*args) == expect
+
+
+def test_fwd_empty_query_is_noop(L):
+    # Lq == 0: valid, nothing to launch
+    assert L.fa_fwd(P16, P16, P16, P16, None, 1, 1, 1, 0, 8, 64, 0.1, 0, None) == fa.FA_OK
+
+
+def test_fwd_ex_bad_dtype(L):
+    assert L.fa_fwd_ex(P16, P16, P16, P16, None, 1, 1, 1, 8, 8, 64, 0.1, 0, 7, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments(L):
+    ws = fa.decode_workspace_size(2, 4, 100, 64)
+    ok = (P16, P16, P16, P16, P16, None, 2, 4, 2, 100, 64, 0.1, 0, 256 * 1024, ws)
+    bad_ws = ok[:-1] + (ws - 1,)
+    assert L.fa_decode_splitkv(*bad_ws, None) == fa.FA_ERR_INVALID_ARG
+    bad_align = ok[:13] + (256 * 1024 + 16, ws)
+    assert L.fa_decode_splitkv(*bad_align, None) == fa.FA_ERR_INVALID_ARG
+    bad_d = ok[:10] + (80,) + ok[11:]
+    assert L.fa_decode_splitkv(*bad_d, None) == fa.FA_ERR_UNSUPPORTED
+    assert L.fa_decode_combine(None, P16, None, P16, None, 1, 1, 64, 2, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_decode_combine(P16, P16, None, P16, None, 1, 1, 64, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_bwd_rejects_bad_arguments(L):
+    ws = fa.bwd_workspace_size(1, 2, 128, 64)
+    base = [P16] * 9 + [1, 2, 2, 128, 128, 64, 0.125, 1, 0, 256 * 1024, ws, None]
+    a = list(base)
+    a[19] = ws - 1
+    assert L.fa_bwd(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(base)
+    a[5] = None                       # lse
+    assert L.fa_bwd(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(base)
+    a[14] = 32
+    assert L.fa_bwd(*a) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_selftest_rejects_bad_limit(L):
+    assert L.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_binding_has_no_cpu_path():
+    import torch
+    q = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        fa.fwd(q, q, q)
