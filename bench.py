@@ -38,6 +38,24 @@ METRIC = "attn fwd/bwd TFLOP/s & % BF16 tensor peak; decode KV-read GB/s & % of 
 HEADLINE = "causal_prefill"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel on the
+# headline workload, valid only while the kernel sources hash to the recorded
+# value (otherwise the roofline's traffic is reported as null).
+PROFILED_TRAFFIC = {
+    "fwd_kernel causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
+                                  "sha256_16": "20c82d9cb46a4479", "bytes": 133.435136e6 + 13.664512e6},
+}
+
+
+def profiled_traffic(key):
+    import hashlib
+    rec = PROFILED_TRAFFIC[key]
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, "exact_tiled_attention_46_b200", rel), "rb") as f:
+            h.update(f.read())
+    return rec["bytes"] if h.hexdigest()[:16] == rec["sha256_16"] else None
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -294,7 +312,7 @@ def run_ours(args):
                    "parallelism": f"replicas{world}", "l2": "flushed (256 MiB write) before every timed step",
                    "flops_per_step": flops, "flop_count": "4*B*H*D*allowed_pairs, causal pairs counted once"},
         "roofline": {"bound": "tensor", "achieved": tf_rank, "peak": peak, "unit": "TFLOP/s",
-                     "frac": tf_rank / peak, "traffic": None, "peak_source": f"{peak_src} bf16 burst",
+                     "frac": tf_rank / peak, "traffic": profiled_traffic("fwd_kernel causal_prefill"), "peak_source": f"{peak_src} bf16 burst",
                      "algorithmic_bytes": fwd_bytes(w)},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,
@@ -370,8 +388,45 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """A few launches of one kernel on one workload, for ncu captures (no timing).
+
+    causal_prefill / long_gqa_prefill / train_fwd_bwd: fa_fwd (and fa_bwd);
+    splitkv_decode_small: split-KV decode on the first 16 sequences of the
+    decode workload (cache 2.1 GB, larger than L2).
+    """
+    import exact_tiled_attention_46_b200 as fa
+    from exact_tiled_attention_46_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    name = args.profile_case
+    if name == "splitkv_decode_small":
+        w = synth.WORKLOADS["splitkv_decode"]
+        B = 16
+        x = synth.decode_inputs(B, w.Hq, w.Hkv, w.Lk, w.D, w.seed, w.len_lo, w.len_hi, device=dev)
+        q, sl = x["q"].to(dev), x["seqlens"].to(dev)
+        for _ in range(args.warmup + args.steps):
+            fa.decode(q, x["k_cache"], x["v_cache"], sl, scale=w.scale)
+    else:
+        w = synth.WORKLOADS[name]
+        x = synth.workload_inputs(w)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        o, lse = fa.fwd(q, k, v, scale=w.scale, causal=w.causal)
+        if w.kind == "train":
+            do = x["do"].to(dev)
+            for _ in range(args.warmup + args.steps):
+                fa.bwd(q, k, v, o, do, lse, scale=w.scale, causal=w.causal)
+        else:
+            for _ in range(args.warmup + args.steps):
+                fa.fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+    torch.cuda.synchronize()
+    print(f"profile case {name}: {args.warmup + args.steps} launches done")
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile-case", default=None,
+                    choices=["causal_prefill", "long_gqa_prefill", "train_fwd_bwd", "splitkv_decode_small"])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
@@ -382,7 +437,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_case:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -207,7 +207,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int nt = n_t[t];
     const float sl2 = p.scale_log2;
     const int row_tile0 = q0 + t * 128;
-    float m_used = -INFINITY, l = 0.f;
+    // l: exact fp32 sum of p (for LSE); lr: sum of the bf16-rounded p that the
+    // P.V product uses (the normaliser of O)
+    float m_used = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
 
     for (int j = 0; j < nt; ++j) {
@@ -233,7 +235,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
       const bool resc = m_tile > m_used + FWD_TAU;   // false while both are -inf
       float alpha = 1.f;
-      if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; m_used = m_tile; }
+      if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; lr *= alpha; m_used = m_tile; }
       if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -245,7 +247,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
       }
       const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-      float ls0 = 0.f, ls1 = 0.f;
+      float ls0 = 0.f, ls1 = 0.f, lr0 = 0.f, lr1 = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -254,12 +256,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           const int c = half * 64 + 2 * i;
           const float p0 = ex2_approx(fmaf(s[c], sl2, -msub));
           const float p1 = ex2_approx(fmaf(s[c + 1], sl2, -msub));
-          ls0 += p0; ls1 += p1;
           pk[i] = pack_bf16x2(p0, p1);
+          ls0 += p0; ls1 += p1;
+          // O's normaliser sums exactly the bf16 values the P.V product uses,
+          // so that O is a normalised weighted average of V rows
+          lr0 += __uint_as_float(pk[i] << 16);
+          lr1 += __uint_as_float(pk[i] & 0xffff0000u);
         }
         tmem_st_32x32b_x32(t_s + half * 32, pk);   // P over the first 64 columns of S
       }
       l += ls0 + ls1;
+      lr += lr0 + lr1;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -269,7 +276,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const bool have_o = ok && nt > 0 && mbar_wait_warp(&o_full[t], 0, lim, W_FWD_O);
     if (have_o) tc_fence_after();
     const bool has = l > 0.f;
-    const float inv_l = has ? 1.f / l : 0.f;
+    const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
     const bool in_range = row < p.Lq;
     if (in_range && p.lse != nullptr)
       p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_used + log2f(l)) * LN2 : -INFINITY;
