@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include <cuda.h>
@@ -111,6 +112,16 @@ fa_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::
   using C = fa::DecCfg<D, GP>;
   if (!ensure_smem_attr(fa::decode_split_kernel<D, GP>, C::SMEM_BYTES, attr_done)) return FA_ERR_CUDA;
   fa::decode_split_kernel<D, GP><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mk, mv, p);
+  return launch_status();
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                     const fa::BwdParams& p, unsigned grid, cudaStream_t st) {
+  static std::atomic<uint64_t> attr_done{0};
+  constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
+  if (!ensure_smem_attr(fa::bwd_main_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
+  fa::bwd_main_kernel<D, CAUSAL><<<grid, fa::BwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, mdo, p);
   return launch_status();
 }
 
@@ -241,14 +252,18 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
 size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D) {
   if (B <= 0 || Hq <= 0 || Lq < 0 || D <= 0) return 0;
   const size_t lq_pad = align_up(size_t(Lq), 128);
-  return align_up(size_t(B) * Lq * Hq * D * 4, 256) + align_up(size_t(B) * Hq * lq_pad * 4, 256);
+  // fp32 dQ accumulator, then the padded log2 LSE and Delta rows
+  return align_up(size_t(B) * Lq * Hq * D * 4, 256) + 2 * align_up(size_t(B) * Hq * lq_pad * 4, 256);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int causal,
                  int grad_dtype, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  // empty tensors may come with null pointers
+  if (Lq > 0 && (!q || !o || !dO || !lse || !dq)) return FA_ERR_INVALID_ARG;
+  if (Lk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  if (Lq > 0 && Lk > 0 && !workspace) return FA_ERR_INVALID_ARG;
   if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
   if (grad_dtype != FA_BF16 && grad_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(dq) ||
@@ -256,9 +271,48 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     return FA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
   if (workspace_bytes < fa_bwd_workspace_size(B, Hq, Lq, D)) return FA_ERR_INVALID_ARG;
-  return fa::bwd_dispatch(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, Lq, Lk, D, scale, causal,
-                          grad_dtype == FA_FP32, workspace, reinterpret_cast<cudaStream_t>(stream),
-                          g_wait_limit_ns.load());
+  if (!fits_int(static_cast<long long>((Lk + 127) / 128) * B * Hkv)) return FA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t g_elt = grad_dtype == FA_FP32 ? 4 : 2;
+  if (Lq == 0 || Lk == 0) {   // no (query, key) pair: the gradients that exist are zero
+    const size_t nk = size_t(B) * Lk * Hkv * D * g_elt, nq = size_t(B) * Lq * Hq * D * g_elt;
+    if ((nk && (cudaMemsetAsync(dk, 0, nk, st) != cudaSuccess || cudaMemsetAsync(dv, 0, nk, st) != cudaSuccess)) ||
+        (nq && cudaMemsetAsync(dq, 0, nq, st) != cudaSuccess))
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  const int lq_pad = static_cast<int>(align_up(size_t(Lq), 128));
+  const size_t acc_bytes = size_t(B) * Lq * Hq * D * 4;
+  const size_t row_bytes = align_up(size_t(B) * Hq * lq_pad * 4, 256);
+  float* dq_acc = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + align_up(acc_bytes, 256));
+  float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + row_bytes);
+  if (cudaMemsetAsync(dq_acc, 0, acc_bytes, st) != cudaSuccess) return FA_ERR_CUDA;
+  {
+    const size_t rows = size_t(B) * lq_pad * Hq;
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 255) / 256, 148 * 16));
+    fa::bwd_pre_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dO),
+                                               lse, lse2, delta, B, Hq, Lq, lq_pad, D);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  CUtensorMap mq, mk, mv, mdo;
+  if (!map_bshd(&mq, q, B, Lq, Hq, D, 64, 128, true) || !map_bshd(&mk, k, B, Lk, Hkv, D, 64, 128, true) ||
+      !map_bshd(&mv, v, B, Lk, Hkv, D, 64, 128, true) || !map_bshd(&mdo, dO, B, Lq, Hq, D, 64, 128, true))
+    return FA_ERR_CUDA;
+  fa::BwdParams p;
+  p.lse2 = lse2; p.delta = delta; p.dq_acc = dq_acc; p.dk = dk; p.dv = dv;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.Lq_pad = lq_pad;
+  p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f; p.g_fp32 = (grad_dtype == FA_FP32);
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const unsigned grid = static_cast<unsigned>(((Lk + 127) / 128) * B * Hkv);
+  fa_status s;
+  if (D == 128) s = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, p, grid, st) : launch_bwd<128, false>(mq, mk, mv, mdo, p, grid, st);
+  else s = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, p, grid, st) : launch_bwd<64, false>(mq, mk, mv, mdo, p, grid, st);
+  if (s != FA_OK) return s;
+  const size_t n = size_t(B) * Lq * Hq * D;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n / 4 + 255) / 256, 148 * 16));
+  fa::bwd_post_kernel<<<blocks, 256, 0, st>>>(dq_acc, dq, n, scale, grad_dtype == FA_FP32);
+  return launch_status();
 }
 
 fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream) {

@@ -1,12 +1,421 @@
-// Backward pass (placeholder until the tcgen05 backward kernels land).
+// Backward pass with the probabilities recomputed from the saved LSE instead
+// of being stored ("FlashAttention Explained: How AI Models Process Attention
+// Faster and Use Less Memory", section "More Efficient Backpropagation"; "How
+// FlashAttention Speeds Up LLM Attention", "Recompute probabilities for
+// training").  With S = scale Q K^T and P = exp(S - LSE):
+//     dV = P^T dO,   dP = dO V^T,   Delta_i = sum_d dO_id O_id,
+//     dS = P * (dP - Delta),   dQ = scale dS K,   dK = scale dS^T Q.
+//
+// Three launches on the caller's stream (plus a memset of the dQ accumulator):
+//   bwd_pre_kernel   Delta, the LSE in log2 units (+inf for rows without a key,
+//                    so that their P is 0), both padded to 128-row tiles.
+//   bwd_main_kernel  one CTA per (batch, kv head, 128-key tile); loops over the
+//                    (query tile, query head of the group) pairs:
+//        warp 8     TMA: K, V once; Q, dO, LSE, Delta per pair (NQ stages)
+//        warp 9     tcgen05: S^T = K Q^T and dP^T = V dO^T into TMEM,
+//                   dV += P^T dO, dK += dS^T Q, dQ = dS K
+//        P^T and dS^T enter the products as bf16.  P^T = P_hi + P_lo and
+//        dS^T = dS_hi + dS_lo (each part bf16; P_hi in TMEM over S^T, the rest
+//        in swizzled shared memory); dV and dK take both parts, so that their
+//        only rounding is the fp32 accumulation, and dQ takes dS_hi.
+//        warps 0-3  one thread per key row: P^T from S^T and the LSE (causal /
+//                   ragged mask), P^T -> TMEM; dS^T = P^T (dP^T - Delta) -> smem
+//        warps 4-7  one thread per query row: dQ tile from TMEM added to the fp32
+//                   accumulator with vector atomics; at the end dK, dV out of TMEM
+//        warp 10    TMEM allocation
+//   bwd_post_kernel  dQ = scale * accumulator, converted to the output dtype.
 #pragma once
 #include "sm100.cuh"
 #include "fa.h"
 
 namespace fa {
-inline fa_status bwd_dispatch(const void*, const void*, const void*, const void*, const void*, const float*, void*,
-                              void*, void*, int, int, int, int, int, int, float, int, bool, void*, cudaStream_t,
-                              uint64_t) {
-  return FA_ERR_UNSUPPORTED;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE = 128 * D * 2;            // 128 rows of bf16
+  static constexpr int NQ = (D == 64) ? 2 : 1;        // Q/dO stages (two do not fit at D = 128)
+  static constexpr int NDS = 1;                       // one set of P_lo / dS_hi / dS_lo buffers
+  static constexpr bool DQ_IN_DP = (D == 128);        // dQ reuses the dP^T columns
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = TILE;
+  static constexpr int Q_OFF = 2 * TILE;              // stage s: Q at +s*2*TILE, dO after it
+  static constexpr int DS_OFF = Q_OFF + NQ * 2 * TILE;
+  static constexpr int DS_BYTES = 128 * 128 * 2;     // one 128 x 128 bf16 operand (128B swizzle)
+  static constexpr int DSLO_OFF = DS_OFF + DS_BYTES;  // low bf16 part of dS^T
+  static constexpr int PLO_OFF = DSLO_OFF + DS_BYTES; // low bf16 part of P^T
+  static constexpr int ROW_OFF = PLO_OFF + DS_BYTES;  // stage s: lse2[128], delta[128]
+  static constexpr int BAR_OFF = ROW_OFF + NQ * 1024;
+  static constexpr int NBARS = 1 + 2 * NQ + 3 + NDS + 4;
+  static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
+  // TMEM columns
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr uint32_t T_DQ = DQ_IN_DP ? T_DP : 256 + 2 * D;
+  static constexpr int THREADS = 384;
+};
+
+struct BwdParams {
+  const float* lse2;     // [B*Hq, Lq_pad]  LSE * log2(e), +inf on rows without keys / padding
+  const float* delta;    // [B*Hq, Lq_pad]
+  float* dq_acc;         // [B, Lq, Hq, D] fp32, zero on entry
+  void* dk;              // [B, Lk, Hkv, D]
+  void* dv;
+  int B, Hq, Hkv, Lq, Lk, Lq_pad;
+  float scale, scale_log2;
+  int g_fp32;
+  uint64_t wait_limit_ns;
+};
+
+enum : uint32_t {
+  W_BWD_KV = 0x301, W_BWD_QF = 0x302, W_BWD_QE = 0x303, W_BWD_SDP = 0x304, W_BWD_P = 0x305,
+  W_BWD_DS = 0x306, W_BWD_DSF = 0x307, W_BWD_DQF = 0x308, W_BWD_DQ = 0x309, W_BWD_DKV = 0x30a,
+  W_BWD_DONE = 0x30b, W_BWD_DRAIN = 0x30c
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Delta = rowsum(dO * O) and the log2-scaled LSE, both padded to Lq_pad rows.
+// Thread per (b, i, h) row with h fastest, so a warp reads neighbouring rows.
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* o, const uint16_t* dO, const float* lse,
+                                                      float* lse2, float* delta, int B, int Hq, int Lq,
+                                                      int Lq_pad, int D) {
+  const size_t n = size_t(B) * Lq_pad * Hq;
+  for (size_t t = blockIdx.x * size_t(blockDim.x) + threadIdx.x; t < n; t += size_t(gridDim.x) * blockDim.x) {
+    const int h = static_cast<int>(t % Hq);
+    const size_t bi = t / Hq;
+    const int i = static_cast<int>(bi % Lq_pad);
+    const int b = static_cast<int>(bi / Lq_pad);
+    const size_t dst = (size_t(b) * Hq + h) * Lq_pad + i;
+    if (i >= Lq) { lse2[dst] = INFINITY; delta[dst] = 0.f; continue; }
+    const size_t row = ((size_t(b) * Lq + i) * Hq + h) * D;
+    const uint4* po = reinterpret_cast<const uint4*>(o + row);
+    const uint4* pd = reinterpret_cast<const uint4*>(dO + row);
+    float acc = 0.f;
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 a = po[c], g = pd[c];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
+        acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(gv[e] & 0xffff0000u), acc);
+      }
+    }
+    const float l = lse[(size_t(b) * Hq + h) * Lq + i];
+    lse2[dst] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    delta[dst] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* acc, void* dq, size_t n, float scale,
+                                                       int g_fp32) {
+  for (size_t t = blockIdx.x * size_t(blockDim.x) + threadIdx.x; t < n / 4; t += size_t(gridDim.x) * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(acc)[t];
+    if (g_fp32) {
+      reinterpret_cast<float4*>(dq)[t] = make_float4(v.x * scale, v.y * scale, v.z * scale, v.w * scale);
+    } else {
+      uint2 w;
+      w.x = pack_bf16x2(v.x * scale, v.y * scale);
+      w.y = pack_bf16x2(v.z * scale, v.w * scale);
+      reinterpret_cast<uint2*>(dq)[t] = w;
+    }
+  }
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int NQ = C::NQ, KB = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = q_full + NQ;
+  uint64_t* sdp_full = q_empty + NQ;
+  uint64_t* p_ready = sdp_full + 1;
+  uint64_t* ds_ready = p_ready + 1;
+  uint64_t* ds_free = ds_ready + 1;
+  uint64_t* dq_full = ds_free + 1;
+  uint64_t* dq_free = dq_full + 1;
+  uint64_t* dkv_done = dq_free + 1;
+  uint64_t* mma_done = dkv_done + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit_ns;
+  const int G = p.Hq / p.Hkv;
+  const int bk = p.B * p.Hkv;
+  const int j = static_cast<int>(blockIdx.x / bk);        // key tile, heaviest (j = 0) first
+  const int b = static_cast<int>(blockIdx.x % bk) / p.Hkv;
+  const int hkv = static_cast<int>(blockIdx.x % bk) % p.Hkv;
+  const int off = p.Lk - p.Lq;
+  const int nq = (p.Lq + 127) >> 7;
+  int i0 = 0;
+  if (CAUSAL) {
+    const int first_q = j * 128 - off;                     // lowest query that sees a key of this tile
+    i0 = first_q <= 0 ? 0 : (first_q >> 7);
+  }
+  const int npairs = (i0 < nq) ? (nq - i0) * G : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < NQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    mbar_init(sdp_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(ds_ready, 128);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(dkv_done, 1);
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 10) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0 && npairs > 0) {
+      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+      for (int kb = 0; kb < KB; ++kb) {
+        tma_load_4d(smem + C::K_OFF + kb * 16384, &tm_k, kv_full, kb * 64, hkv, j * 128, b);
+        tma_load_4d(smem + C::V_OFF + kb * 16384, &tm_v, kv_full, kb * 64, hkv, j * 128, b);
+      }
+      int issued = 0;
+      for (int n = 0; n < npairs; ++n) {
+        const int s = n % NQ;
+        if (n >= NQ && !mbar_wait(&q_empty[s], ((n / NQ) + 1) & 1, lim, W_BWD_QE)) break;
+        const int i = i0 + n / G, hq = hkv * G + n % G;
+        mbar_arrive_expect_tx(&q_full[s], 2 * C::TILE + 1024);
+        uint8_t* qdst = smem + C::Q_OFF + s * 2 * C::TILE;
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_4d(qdst + kb * 16384, &tm_q, &q_full[s], kb * 64, hq, i * 128, b);
+          tma_load_4d(qdst + C::TILE + kb * 16384, &tm_do, &q_full[s], kb * 64, hq, i * 128, b);
+        }
+        const size_t rowbase = (size_t(b) * p.Hq + hq) * p.Lq_pad + size_t(i) * 128;
+        float* rdst = reinterpret_cast<float*>(smem + C::ROW_OFF + s * 1024);
+        bulk_load(rdst, p.lse2 + rowbase, 512, &q_full[s]);
+        bulk_load(rdst + 128, p.delta + rowbase, 512, &q_full[s]);
+        issued = n + 1;
+      }
+      mbar_wait(kv_full, 0, lim, W_BWD_DRAIN);
+      for (int n = max(0, issued - NQ); n < issued; ++n) mbar_wait(&q_full[n % NQ], (n / NQ) & 1, lim, W_BWD_DRAIN);
+    }
+  } else if (warp == 9) {
+    // ----------------------------------------------------------------- MMA --
+    if (lane == 0 && npairs > 0) {
+      constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t ID_DVK = idesc_bf16_f32(128, D, false, true);     // dV, dK: B = dO / Q (MN-major)
+      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, true, true);       // dQ: A = dS (MN-major), B = K (MN-major)
+      const uint32_t k_base = smem_u32(smem + C::K_OFF), v_base = smem_u32(smem + C::V_OFF);
+      const uint32_t q_base = smem_u32(smem + C::Q_OFF), ds_base = smem_u32(smem + C::DS_OFF);
+      const uint32_t dslo_base = smem_u32(smem + C::DSLO_OFF), plo_base = smem_u32(smem + C::PLO_OFF);
+      auto kmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
+      auto mnmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + kk * 2048, 16384, 1024); };
+      auto issue_s_dp = [&](int n) {
+        const uint32_t qa = q_base + (n % NQ) * 2 * C::TILE, da = qa + C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_S, kmaj(k_base, kk), kmaj(qa, kk), ID_SS, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_DP, kmaj(v_base, kk), kmaj(da, kk), ID_SS, kk > 0);
+      };
+      bool ok = mbar_wait(kv_full, 0, lim, W_BWD_KV) && mbar_wait(&q_full[0], 0, lim, W_BWD_QF);
+      tc_fence_after();
+      if (ok) { issue_s_dp(0); umma_commit(sdp_full); }
+      for (int n = 0; ok && n < npairs; ++n) {
+        const int s = n % NQ;
+        const uint32_t qa = q_base + s * 2 * C::TILE, da = qa + C::TILE;
+        const uint32_t dsa = ds_base;
+        if (!(ok = mbar_wait(p_ready, n & 1, lim, W_BWD_P))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // dV += P_hi^T dO  (K = 128 queries)
+          umma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
+        if (!(ok = mbar_wait(ds_ready, n & 1, lim, W_BWD_DS))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // dV += P_lo^T dO
+          umma_ss(tmem + C::T_DV, kmaj(plo_base, kk), mnmaj(da, kk), ID_DVK, 1u);
+        const bool more = n + 1 < npairs;
+        if (!C::DQ_IN_DP && more) {         // next pair's S^T, dP^T first: the softmax warps start early
+          if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
+          tc_fence_after();
+          issue_s_dp(n + 1);
+          umma_commit(sdp_full);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // dK += dS_hi^T Q  (K = 128 queries)
+          umma_ss(tmem + C::T_DK, kmaj(dsa, kk), mnmaj(qa, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // dK += dS_lo^T Q
+          umma_ss(tmem + C::T_DK, kmaj(dslo_base, kk), mnmaj(qa, kk), ID_DVK, 1u);
+        if (!C::DQ_IN_DP && n > 0) {        // dQ(n-1) must have been read out of TMEM
+          if (!(ok = mbar_wait(dq_free, (n - 1) & 1, lim, W_BWD_DQF))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)      // dQ = dS K  (K = 128 keys)
+          umma_ss(tmem + C::T_DQ, mnmaj(dsa, kk), mnmaj(k_base, kk), ID_DQ, kk > 0 ? 1u : 0u);
+        umma_commit(dq_full);
+        umma_commit(ds_free);
+        umma_commit(&q_empty[s]);
+        if (C::DQ_IN_DP && more) {          // dP^T(n+1) overwrites dQ(n): wait for its read-out
+          if (!(ok = mbar_wait(dq_free, n & 1, lim, W_BWD_DQF))) break;
+          if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
+          tc_fence_after();
+          issue_s_dp(n + 1);
+          umma_commit(sdp_full);
+        }
+      }
+      umma_commit(dkv_done);
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, lim, W_BWD_DONE);
+    }
+  } else if (warp < 4) {
+    // --------------------------------------------- P^T and dS^T (key rows) --
+    const int r = warp * 32 + lane;
+    const int key = j * 128 + r;
+    const bool key_ok = key < p.Lk;
+    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    for (int n = 0; n < npairs; ++n) {
+      const int s = n % NQ;
+      const int i = i0 + n / G;
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::ROW_OFF + s * 1024);
+      const float* dlt = lse2 + 128;
+      if (!mbar_wait_warp(sdp_full, n & 1, lim, W_BWD_SDP)) break;
+      tc_fence_after();
+      // allowed when key <= query + off, i.e. column c >= cmin
+      const int cmin = CAUSAL ? key - off - i * 128 : -1;
+      const int rowoff = r * 128;
+      bool ok = true;
+      // 32 query columns per step.  P_hi (bf16) of columns [32ch, 32ch+32) goes to
+      // TMEM columns [16ch, 16ch+16) of the S^T block, below every S^T column
+      // still to be read; P_lo, dS_hi and dS_lo go to shared memory.
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dp[32];
+        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_S + ch * 32, sv);
+        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DP + ch * 32, dp);
+        uint32_t phi[16], plo[16], dhi[16], dlo[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int c = ch * 32 + 2 * t;
+          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + c);
+          const float2 d2 = *reinterpret_cast<const float2*>(dlt + c);
+          float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, -l2.x));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, -l2.y));
+          p0 = (key_ok && c >= cmin) ? p0 : 0.f;
+          p1 = (key_ok && c + 1 >= cmin) ? p1 : 0.f;
+          phi[t] = pack_bf16x2(p0, p1);
+          plo[t] = pack_bf16x2(p0 - __uint_as_float(phi[t] << 16), p1 - __uint_as_float(phi[t] & 0xffff0000u));
+          const float s0 = p0 * (__uint_as_float(dp[2 * t]) - d2.x);
+          const float s1 = p1 * (__uint_as_float(dp[2 * t + 1]) - d2.y);
+          dhi[t] = pack_bf16x2(s0, s1);
+          dlo[t] = pack_bf16x2(s0 - __uint_as_float(dhi[t] << 16), s1 - __uint_as_float(dhi[t] & 0xffff0000u));
+        }
+        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + ch * 16, phi);
+        // the shared-memory operands of pair n - 1 must have been consumed
+        if (ch == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
+        // 32 columns = 4 16-byte chunks of the 128-byte row of block ch/2 (128B swizzle)
+        const int blk = (ch >> 1) * 16384 + rowoff;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int o16 = blk + ((((ch & 1) * 4 + t) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(smem + C::PLO_OFF + o16) = make_uint4(plo[4 * t], plo[4 * t + 1], plo[4 * t + 2], plo[4 * t + 3]);
+          *reinterpret_cast<uint4*>(smem + C::DS_OFF + o16) = make_uint4(dhi[4 * t], dhi[4 * t + 1], dhi[4 * t + 2], dhi[4 * t + 3]);
+          *reinterpret_cast<uint4*>(smem + C::DSLO_OFF + o16) = make_uint4(dlo[4 * t], dlo[4 * t + 1], dlo[4 * t + 2], dlo[4 * t + 3]);
+        }
+      }
+      if (!ok) break;
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      mbar_arrive(ds_ready);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------- dQ read-out, then dK/dV epilogue --
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = true;
+    for (int n = 0; n < npairs; ++n) {
+      if (!(ok = mbar_wait_warp(dq_full, n & 1, lim, W_BWD_DQ))) break;
+      tc_fence_after();
+      const int i = i0 + n / G, hq = hkv * G + n % G;
+      const int qrow = i * 128 + r;
+      float* dst = p.dq_acc + ((size_t(b) * p.Lq + qrow) * p.Hq + hq) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DQ + c0, v);
+        if (qrow < p.Lq) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            atomicAdd(reinterpret_cast<float4*>(dst + c0) + t,
+                      make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                                  __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
+    const bool have = ok && npairs > 0 && mbar_wait_warp(dkv_done, 0, lim, W_BWD_DKV);
+    if (have) tc_fence_after();
+    const int key = j * 128 + r;
+    const size_t krow = ((size_t(b) * p.Lk + key) * p.Hkv + hkv) * D;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {       // 0: dV, 1: dK (scaled)
+      const float mul = which ? p.scale : 1.f;
+      void* out = which ? p.dk : p.dv;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld_32x32b_x32(tmem + lane_bits + (which ? C::T_DK : C::T_DV) + c0, v);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = 0u;
+        }
+        if (key >= p.Lk) continue;
+        if (p.g_fp32) {
+          float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(out) + krow + c0);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            d4[t] = make_float4(__uint_as_float(v[4 * t]) * mul, __uint_as_float(v[4 * t + 1]) * mul,
+                                __uint_as_float(v[4 * t + 2]) * mul, __uint_as_float(v[4 * t + 3]) * mul);
+        } else {
+          uint4* d4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + krow + c0);
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            d4[t] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * t]) * mul, __uint_as_float(v[8 * t + 1]) * mul),
+                               pack_bf16x2(__uint_as_float(v[8 * t + 2]) * mul, __uint_as_float(v[8 * t + 3]) * mul),
+                               pack_bf16x2(__uint_as_float(v[8 * t + 4]) * mul, __uint_as_float(v[8 * t + 5]) * mul),
+                               pack_bf16x2(__uint_as_float(v[8 * t + 6]) * mul, __uint_as_float(v[8 * t + 7]) * mul));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 10) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace fa

@@ -1,0 +1,79 @@
+"""Backward kernels vs the CPU fp64 oracle gradients (GPU)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import exact_tiled_attention_46_b200 as fa
+from exact_tiled_attention_46_b200 import inputs as synth
+
+from parity import check_close, need_gpu, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def gpu_grads(x, scale, causal, grad_dtype):
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.fwd(q, k, v, scale=scale, causal=causal)
+    dq, dk, dv = fa.bwd(q, k, v, o, do, lse, scale=scale, causal=causal, grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    return f64(dq), f64(dk), f64(dv)
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, Lk, D, causal
+    (1, 2, 2, 128, 128, 64, True),
+    (1, 2, 1, 200, 200, 64, True),
+    (2, 4, 2, 255, 255, 64, False),
+    (1, 2, 2, 384, 384, 64, True),
+    (1, 4, 1, 256, 512, 64, True),      # Lq < Lk
+    (1, 2, 2, 300, 100, 64, True),      # Lq > Lk: queries without keys
+    (1, 2, 2, 300, 300, 128, True),
+    (1, 4, 2, 129, 257, 128, False),
+    (1, 1, 1, 1, 1, 64, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dHq%dHkv%dLq%dLk%dD%d%s" % (*c[:6], "c" if c[6] else "n"))
+def test_bwd_matches_oracle(case):
+    B, Hq, Hkv, Lq, Lk, D, causal = case
+    x = synth.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=sum(case) + 7, with_do=True)
+    scale = 1.0 / math.sqrt(D)
+    xf = {n: synth.as_f64(x[n]) for n in x}
+    rq, rk, rv, *_ = oracle.attn_bwd(xf["q"], xf["k"], xf["v"], xf["do"], scale, causal)
+    for gdt in (torch.float32, torch.bfloat16):
+        dq, dk, dv = gpu_grads(x, scale, causal, gdt)
+        bf = gdt == torch.bfloat16
+        check_close(dv, rv, bf16_output=bf, what=f"dV {gdt}")
+        check_close(dk, rk, bf16_output=bf, what=f"dK {gdt}")
+        check_close(dq, rq, bf16_output=bf, what=f"dQ {gdt}")
+
+
+def test_bwd_empty_queries():
+    k = torch.randn(1, 64, 2, 64, device="cuda").to(torch.bfloat16)
+    q = torch.empty(1, 0, 2, 64, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(1, 2, 0, device="cuda")
+    dq, dk, dv = fa.bwd(q, k, k, q, q, lse, causal=False)
+    torch.cuda.synchronize()
+    assert torch.all(dk == 0) and torch.all(dv == 0) and dq.numel() == 0
+
+
+def test_bwd_training_workload_sampled_heads():
+    """B8 H16 L4096 D64 causal fwd+bwd (seed 3): whole heads checked against the oracle."""
+    w = synth.WORKLOADS["train_fwd_bwd"]
+    x = synth.workload_inputs(w)
+    dq, dk, dv = gpu_grads(x, w.scale, w.causal, torch.float32)
+    xf = {n: synth.as_f64(x[n]) for n in x}
+    for b, h in [(0, 0), (3, 9), (7, 15)]:
+        sl = lambda t: t[b:b + 1, :, h:h + 1]
+        rq, rk, rv, *_ = oracle.attn_bwd(sl(xf["q"]), sl(xf["k"]), sl(xf["v"]), sl(xf["do"]), w.scale, w.causal)
+        check_close(sl(dv), rv, bf16_output=False, what=f"dV b{b} h{h}")
+        check_close(sl(dk), rk, bf16_output=False, what=f"dK b{b} h{h}")
+        check_close(sl(dq), rq, bf16_output=False, what=f"dQ b{b} h{h}")
