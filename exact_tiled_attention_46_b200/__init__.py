@@ -39,6 +39,7 @@ _SIGNATURES = {
     "fa_decode_workspace_size": ([_i, _i, _i, _i], _sz),
     "fa_decode_splitkv": ([_vp] * 6 + [_i] * 5 + [_f, _i, _vp, _sz, _vp], _i),
     "fa_decode_combine": ([_vp] * 5 + [_i] * 5 + [_vp], _i),
+    "fa_decode_splitkv_static": ([_vp] * 6 + [_i] * 5 + [_f, _i, _vp], _i),
     "fa_device_status": ([ctypes.POINTER(_i), ctypes.POINTER(_i), _i, _vp], _i),
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
     "fa_selftest_wait_timeout": ([ctypes.c_ulonglong, _vp], _i),

@@ -125,6 +125,13 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return launch_status();
 }
 
+// Scratch of fa_decode_splitkv_static: the split-KV partial results of the
+// most recent call.  In host code this name is only a stand-in for the device
+// array; its device address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_decode_static_scratch[FA_DECODE_STATIC_SCRATCH_BYTES];
+std::mutex g_static_mu;
+void* g_static_scratch_ptr[64] = {};
+
 }  // namespace
 
 extern "C" {
@@ -247,6 +254,27 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
   c.B = B; c.Hq = Hq; c.D = D; c.max_splits = max_splits; c.chunk = kDecodeChunk; c.o_fp32 = (o_dtype == FA_FP32);
   fa::decode_combine_kernel<<<B * Hq, 128, 0, st>>>(c);
   return launch_status();
+}
+
+fa_status fa_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
+                                   void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                                   int o_dtype, fa_stream_t stream) {
+  if (fa_decode_workspace_size(B, Hq, Lmax, D) > FA_DECODE_STATIC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    // set-up, once per device, with that device current
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_scratch_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_decode_static_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+      g_static_scratch_ptr[dev] = ptr;
+    }
+    scratch = g_static_scratch_ptr[dev];
+  }
+  return fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, B, Hq, Hkv, Lmax, D, scale, o_dtype, scratch,
+                           FA_DECODE_STATIC_SCRATCH_BYTES, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D) {

@@ -112,6 +112,38 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
                             fa_stream_t stream);
 
 /*
+ * Split-KV decode that allocates nothing and takes no workspace.  The pages
+ * have no counterpart to this entry point; it exists for callers that cannot
+ * obtain device memory at the moment they run a decode step: for example an
+ * engine plugin or serving loop whose memory is fixed when it starts and that
+ * may not call cudaMalloc later (cudaMalloc can block and synchronise the
+ * device, which a per-token latency budget cannot absorb), or a foreign-
+ * language caller that can only hand over the tensors it already owns.
+ *
+ * Arguments, layouts and results are those of fa_decode_splitkv without the
+ * workspace pair; the caller still owns and passes every input and output.
+ * The partial results live instead in one file-scope device array of
+ * FA_DECODE_STATIC_SCRATCH_BYTES bytes inside the library.  Every GPU that
+ * loads the library holds that array until the process exits.  A
+ * configuration whose fa_decode_workspace_size() exceeds it returns
+ * FA_ERR_UNSUPPORTED and launches nothing.
+ *
+ * The first call on a device looks up the array's address on that device
+ * (with that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents; nothing
+ * in it has to start at zero, because every partial result the combine step
+ * reads is written earlier in the same call.  Calls whose kernels may overlap
+ * on the GPU (different streams, or threads without ordering between them)
+ * race on the array and corrupt each other's results: order such calls.
+ * Never calls cudaMalloc, cudaFree or any allocating library routine.
+ */
+#define FA_DECODE_STATIC_SCRATCH_BYTES (40u * 1024u * 1024u)
+fa_status fa_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache,
+                                   const int* seqlens, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                                   int o_dtype, fa_stream_t stream);
+
+/*
  * Combine partial results over disjoint key sets (the merge step of split-KV
  * decode; "How FlashAttention Speeds Up LLM Attention": partial results kept
  * on the same numerical scale).  o_part [B,Hq,max_splits,D] fp32 holds
