@@ -128,6 +128,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
+# ------------------------------------------------------- rank helpers ------
+def max_over_ranks(ms, dist=None, device="cpu"):
+    """Device time of the slowest rank (the whole job ends when it does)."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, world, steps, max_ms):
+    """Replicas: every rank runs the same workload, so the job did world x steps of it."""
+    return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------- our arm -----
 def l2_flusher(dev):
     buf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -258,14 +272,10 @@ def run_ours(args):
     if dist:
         dist.barrier()
     ck = clocks.stop() if rank == 0 else None
-    kernel_ms = sum(s.elapsed_time(e) for s, e in evs)
-    t_local = torch.tensor([kernel_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    kernel_ms = float(t_local.item())
+    kernel_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in evs), dist, dev)
     ms_step = kernel_ms / args.steps
     flops = fwd_flops(w)
-    value = flops * world * args.steps / (kernel_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, args.steps, kernel_ms)
     tf_rank = flops / (ms_step * 1e-3) / 1e12
 
     # end to end through the public API: pinned host inputs -> device -> fwd -> host
