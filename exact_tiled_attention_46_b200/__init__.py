@@ -43,6 +43,7 @@ _SIGNATURES = {
     "fa_device_status": ([ctypes.POINTER(_i), ctypes.POINTER(_i), _i, _vp], _i),
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
     "fa_selftest_wait_timeout": ([ctypes.c_ulonglong, _vp], _i),
+    "fa_selftest_exp2_poly": ([_vp, _vp, _i, _vp], _i),
 }
 
 _lib = None

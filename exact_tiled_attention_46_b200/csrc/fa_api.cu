@@ -95,11 +95,38 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   fa::mbar_wait(&bar, 0, limit_ns, 0x9001);   // no thread ever arrives
 }
 
+__global__ void selftest_exp2_poly_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    fa::exp2_poly2(x[i], x[i + 1], y[i], y[i + 1]);
+  } else if (i < n) {
+    float unused;
+    fa::exp2_poly2(x[i], x[i], y[i], unused);
+  }
+}
+
+// The forward kernel moves registers between warpgroups (setmaxnreg); that is
+// only safe when the launch allocation per thread is exactly the one the split
+// was computed for.  A build that allocates differently is refused, never run.
+template <typename F>
+bool launch_regs_match(F* func, int expected) {
+  static std::atomic<int> state{0};   // 0 unknown, 1 match, 2 mismatch
+  int s = state.load();
+  if (s == 0) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, func) != cudaSuccess) return false;
+    s = (a.numRegs == expected) ? 1 : 2;
+    state.store(s);
+  }
+  return s == 1;
+}
+
 template <int D, bool CAUSAL>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      long long grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int smem = fa::FwdCfg<D>::SMEM_BYTES;
+  if (!launch_regs_match(fa::fwd_kernel<D, CAUSAL>, fa::FWD_LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(fa::fwd_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
   fa::fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), fa::FwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, p);
   return launch_status();
@@ -360,6 +387,14 @@ fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream)
       return FA_ERR_CUDA;
   }
   return FA_OK;
+}
+
+fa_status fa_selftest_exp2_poly(const float* x, float* y, int n, fa_stream_t stream) {
+  if (!x || !y || n < 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  const int threads = 256, pairs = (n + 1) / 2;
+  selftest_exp2_poly_kernel<<<(pairs + threads - 1) / threads, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
 }
 
 fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t stream) {

@@ -14,10 +14,16 @@
 //               running sum l in log2 units; P (bf16) written over S in TMEM;
 //               O rescaled in TMEM only when the max grows by more than TAU;
 //               epilogue O / l and LSE.
-//   warp 10     allocates / frees the 512 TMEM columns.
+//   warp 10     allocates / frees the 512 TMEM columns; warp 11 idles.
+// Registers: the block is launched with FWD_LAUNCH_REGS per thread (3 warps per
+// SM sub-partition); the control warpgroup (warps 8-11) gives registers back
+// (setmaxnreg.dec to FWD_CTRL_REGS) and the two softmax warpgroups take them
+// (setmaxnreg.inc to FWD_SOFTMAX_REGS).  The split sums to exactly the launch
+// allocation: 2 * 224 + 56 = 3 * 168 registers per lane slot.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 #pragma once
 #include "sm100.cuh"
+#include "exp2_poly.cuh"
 
 namespace fa {
 
@@ -43,9 +49,38 @@ struct FwdCfg {
   static constexpr int THREADS = 384;
 };
 
-// rescale O only when the running max grows by more than 2^8 (log2 units);
-// otherwise the stale max stays the reference and P <= 2^8.
+// The running max m is a reference only: any m gives the same exact result.
+// A tile is first exponentiated against the current m; if no lane's tile sum
+// exceeds 2^FWD_FAST_LOG2 (so every p <= 2^16, a range bf16 and the fp32
+// accumulators hold with unchanged relative precision), that is the tile's P.
+// Otherwise (and on a row's first tile) the tile max is taken, m moves to it
+// when it grows by more than FWD_TAU, O and the sums are rescaled in place, and
+// P is recomputed.
 constexpr float FWD_TAU = 8.0f;
+constexpr int FWD_LAUNCH_REGS = 168, FWD_SOFTMAX_REGS = 224, FWD_CTRL_REGS = 56;
+static_assert(2 * FWD_SOFTMAX_REGS + FWD_CTRL_REGS == 3 * FWD_LAUNCH_REGS, "register split must match the launch");
+constexpr float FWD_FAST_LIMIT = 65536.0f;
+
+// 2^x for two lanes on the FMA pipe: x = j + f with j = round(x), f in
+// [-1/2, 1/2]; 2^f by the fitted polynomial (exp2_poly.cuh, Horner on packed
+// fp32); 2^j added into the exponent field.  x is clamped at -126, so the result
+// is a tiny positive number (not 0) far below 2^-126: callers use it only where
+// no entry is masked.  Relative error <= FA_EXP2_MAX_REL_ERR + fp32 rounding.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  constexpr float RND = 12582912.f;                  // 1.5 * 2^23: x + RND rounds x to an integer
+  float t0, t1, r0, r1, f0, f1, q0, q1;
+  fadd2(t0, t1, x0, x1, RND, RND);
+  fadd2(r0, r1, t0, t1, -RND, -RND);                 // round(x) as a float
+  ffma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);         // f = x - round(x)
+  ffma2(q0, q1, f0, f1, FA_EXP2_C3, FA_EXP2_C3, FA_EXP2_C2, FA_EXP2_C2);
+  ffma2(q0, q1, q0, q1, f0, f1, FA_EXP2_C1, FA_EXP2_C1);
+  ffma2(q0, q1, q0, q1, f0, f1, FA_EXP2_C0, FA_EXP2_C0);
+  // the low mantissa bits of t hold round(x) (two's complement); << 23 moves it to the exponent
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
 
 enum : uint32_t {
   W_FWD_Q = 0x101, W_FWD_KV_EMPTY = 0x102, W_FWD_KV_FULL = 0x103, W_FWD_P = 0x104,
@@ -113,6 +148,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  if (warp >= 8) {
+  setmaxnreg_dec<FWD_CTRL_REGS>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
     if (lane == 0 && n > 0) {
@@ -196,7 +233,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, lim, W_FWD_DONE);
     }
-  } else if (warp < 8) {
+  }
+  // Take the launch budget back only after the softmax warps have returned
+  // theirs (named barrier 2): re-acquiring earlier could starve a softmax warp
+  // that has not yet grown, and both would wait forever.
+  asm volatile("bar.sync 2, %0;" :: "n"(FwdCfg<D>::THREADS) : "memory");
+  setmaxnreg_inc<FWD_LAUNCH_REGS>();
+  } else {
+    setmaxnreg_inc<FWD_SOFTMAX_REGS>();
     // ------------------------------------------------------------- softmax --
     const int t = warp >> 2;
     const int wq = warp & 3;                       // TMEM lane quadrant of this warp
@@ -226,44 +270,61 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = (c < lim_c) ? s[c] : -INFINITY;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]); mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      const bool resc = m_tile > m_used + FWD_TAU;   // false while both are -inf
-      float alpha = 1.f;
-      if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; lr *= alpha; m_used = m_tile; }
-      if (j > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t ov[32];
-          tmem_ld_32x32b_x32(t_o + c0, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st_32x32b_x32(t_o + c0, ov);
-        }
-      }
-      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
       float ls0 = 0.f, ls1 = 0.f, lr0 = 0.f, lr1 = 0.f;
+      // P = 2^(s*scale*log2e - m), packed to bf16 and stored over the first 64
+      // columns of S; ls = exact sum, lr = sum of the bf16 values (O's normaliser)
+      auto exp_tile = [&](float msub, bool use_poly) {
+        ls0 = ls1 = lr0 = lr1 = 0.f;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = half * 64 + 2 * i;
-          const float p0 = ex2_approx(fmaf(s[c], sl2, -msub));
-          const float p1 = ex2_approx(fmaf(s[c + 1], sl2, -msub));
-          pk[i] = pack_bf16x2(p0, p1);
-          ls0 += p0; ls1 += p1;
-          // O's normaliser sums exactly the bf16 values the P.V product uses,
-          // so that O is a normalised weighted average of V rows
-          lr0 += __uint_as_float(pk[i] << 16);
-          lr1 += __uint_as_float(pk[i] & 0xffff0000u);
+          for (int i = 0; i < 32; ++i) {
+            const int c = half * 64 + 2 * i;
+            float x0, x1, p0, p1;
+            ffma2(x0, x1, s[c], s[c + 1], sl2, sl2, -msub, -msub);
+            if (use_poly && (i % 3) == 2) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            pk[i] = pack_bf16x2(p0, p1);
+            fadd2(ls0, ls1, ls0, ls1, p0, p1);
+            add_bf16x2_f32(lr0, lr1, pk[i]);
+          }
+          tmem_st_32x32b_x32(t_s + half * 32, pk);
         }
-        tmem_st_32x32b_x32(t_s + half * 32, pk);   // P over the first 64 columns of S
+      };
+      bool slow = __any_sync(0xffffffffu, m_used == -INFINITY);
+      if (!slow) {
+        // the branch keeps the polynomial loop and the all-MUFU loop apart, so
+        // that the compiler cannot evaluate both and select
+        if (need_mask) exp_tile(m_used, false);
+        else exp_tile(m_used, true);
+        slow = __any_sync(0xffffffffu, !(ls0 + ls1 <= FWD_FAST_LIMIT));
+      }
+      if (slow) {
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]); mx2 = fmaxf(mx2, s[c + 2]); mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        const bool resc = m_tile > m_used + FWD_TAU;   // false while both are -inf
+        float alpha = 1.f;
+        if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; lr *= alpha; m_used = m_tile; }
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(t_o + c0, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st_32x32b_x32(t_o + c0, ov);
+          }
+        }
+        exp_tile((m_used == -INFINITY) ? 0.f : m_used, false);
       }
       l += ls0 + ls1;
       lr += lr0 + lr1;
@@ -310,6 +371,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
       }
     }
+    setmaxnreg_dec<FWD_LAUNCH_REGS>();    // give the extra registers back first
+    asm volatile("bar.arrive 2, %0;" :: "n"(FwdCfg<D>::THREADS) : "memory");
   }
 
   tc_fence_before();
