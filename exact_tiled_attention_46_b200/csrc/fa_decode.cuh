@@ -8,8 +8,8 @@
 // (sequence, kv head, chunk) and the GP query heads of that kv head that it
 // packs, so each K/V byte is read from HBM once for GP heads.  Warp 4 streams
 // K and V tiles of T keys with TMA through an NS-slot mbarrier ring; warps 0-3
-// split every tile's keys, LPK lanes per key, each lane owning 16 of the D
-// dimensions.  Each key group keeps its own running max / running sum /
+// split every tile's keys, LPK = D/8 lanes per key, each lane owning 8
+// consecutive dimensions (one 16-byte chunk of a row).  Each key group keeps its own running max / running sum /
 // accumulator (log2 units); at the end of the chunk the groups and warps are
 // merged and the chunk's normalised partial output and LSE are written.  The
 // combine kernel merges the chunks of a sequence:
@@ -34,7 +34,7 @@ struct DecCfg {
   static constexpr int T = 32;                  // keys per TMA box
   static constexpr int NS = 4;                  // ring slots (K and V tile each)
   static constexpr int NW = 4;                  // consumer warps
-  static constexpr int LPK = D / 16;            // lanes per key
+  static constexpr int LPK = D / 8;             // lanes per key (8 dimensions each)
   static constexpr int KPW = 32 / LPK;          // keys per warp step
   static constexpr int TILE_BYTES = T * D * 2;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -56,8 +56,39 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
   f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
 }
 
+// Sums each of the GP partial dot products over the LPK lanes of a key group
+// and leaves every lane with all GP totals.  For GP = 4 and LPK = 8 the sums
+// are transposed while they are reduced (lane bits 2 and 1 pick which heads a
+// lane keeps), so that 4 shuffles + 4 adds give each lane one head's total and
+// 3 more shuffles collect the other three.
+template <int GP, int LPK>
+__device__ __forceinline__ void reduce_scores(float (&sc)[GP], int lane) {
+  if constexpr (GP == 4 && (LPK == 8 || LPK == 16)) {
+    // the two highest lane bits of the group (H = LPK/2, H/2) choose the kept head
+    constexpr int H = LPK / 2;
+    const bool bh = lane & H, bl = lane & (H / 2);
+    float k0 = bh ? sc[2] : sc[0], k1 = bh ? sc[3] : sc[1];
+    const float s0 = bh ? sc[0] : sc[2], s1 = bh ? sc[1] : sc[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, H);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, H);
+    float kept = bl ? k1 : k0;
+    kept += __shfl_xor_sync(0xffffffffu, bl ? k0 : k1, H / 2);
+#pragma unroll
+    for (int o = H / 4; o >= 1; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+    // lane holds head (bh, bl) summed over the group; collect all four
+    const int base = lane & ~(LPK - 1);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) sc[g] = __shfl_sync(0xffffffffu, kept, base + g * (H / 2));
+  } else {
+#pragma unroll
+    for (int o = 1; o < LPK; o <<= 1)
+#pragma unroll
+      for (int g = 0; g < GP; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], o);
+  }
+}
+
 template <int D, int GP>
-__global__ void __launch_bounds__(DecCfg<D, GP>::THREADS)
+__global__ void __launch_bounds__(DecCfg<D, GP>::THREADS, 3)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const DecParams p) {
   using C = DecCfg<D, GP>;
@@ -109,67 +140,86 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   // -------------------------------------------------------------- consumers --
   const int kg = lane / LPK;                    // key slot within a warp step
-  const int ds = lane % LPK;                    // d-slice: 16B chunks ds and ds + LPK
-  float qf[GP][16];
+  const int ds = lane % LPK;                    // 16-byte chunk: dimensions 8*ds .. 8*ds+7
+  float qf[GP][8];
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
     const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq0 + g) * D);
     bf16x8_to_f32(qrow[ds], qf[g]);
-    bf16x8_to_f32(qrow[ds + LPK], qf[g] + 8);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) qf[g][e] *= p.scale_log2;
+    for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;
   }
-  float m[GP], l[GP], acc[GP][16];
+  float m[GP], l[GP], acc[GP][8];
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
     m[g] = -INFINITY; l[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) acc[g][e] = 0.f;
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
   }
 
+  // Per tile, a lane group owns KS keys (kt = warp*T/NW + st*KPW + kg).  Their
+  // scores are formed first (independent, so their reductions overlap), then
+  // one tile max per head decides a (rare) rescale, then p and the P.V update.
+  constexpr int KS = (T / NW) / KPW;
   bool ok = true;
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % NS;
     if (!(ok = mbar_wait(&full[s], (i / NS) & 1, lim, W_DEC_FULL))) break;
     const uint8_t* ks = smem + s * C::STAGE_BYTES;
     const uint8_t* vs = ks + C::TILE_BYTES;
+    const int key0 = k_begin + i * T;
+    const bool full_tile = key0 + T <= k_end;
+    float sc[KS][GP];
 #pragma unroll
-    for (int step = 0; step < (T / NW) / KPW; ++step) {
-      const int kt = warp * (T / NW) + step * KPW + kg;
-      const bool valid = k_begin + i * T + kt < k_end;
-      float kf[16];
+    for (int st = 0; st < KS; ++st) {
+      const int kt = warp * (T / NW) + st * KPW + kg;
+      float kf[8];
       bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + kt * D * 2 + ds * 16), kf);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + kt * D * 2 + (ds + LPK) * 16), kf + 8);
-      float sc[GP];
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) { a0 = fmaf(qf[g][e], kf[e], a0); a1 = fmaf(qf[g][e + 1], kf[e + 1], a1); }
-        sc[g] = a0 + a1;
+        for (int e = 0; e < 8; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1], a0, a1);
+        sc[st][g] = a0 + a1;
       }
+    }
 #pragma unroll
-      for (int o = 1; o < LPK; o <<= 1)
+    for (int st = 0; st < KS; ++st) reduce_scores<GP, LPK>(sc[st], lane);
+    if (!full_tile) {                             // keys past the chunk end do not count
 #pragma unroll
-        for (int g = 0; g < GP; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], o);
-      float vf[16];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + kt * D * 2 + ds * 16), vf);
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + kt * D * 2 + (ds + LPK) * 16), vf + 8);
-      if (valid) {
+      for (int st = 0; st < KS; ++st) {
+        const int kt = warp * (T / NW) + st * KPW + kg;
+        if (key0 + kt >= k_end) {
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          if (sc[g] > m[g] + DEC_TAU) {
-            const float a = ex2_approx(m[g] - sc[g]);
-            l[g] *= a;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) acc[g][e] *= a;
-            m[g] = sc[g];
-          }
-          const float pr = ex2_approx(sc[g] - m[g]);
-          l[g] += pr;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) acc[g][e] = fmaf(pr, vf[e], acc[g][e]);
+          for (int g = 0; g < GP; ++g) sc[st][g] = -INFINITY;
         }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float mt = sc[0][g];
+#pragma unroll
+      for (int st = 1; st < KS; ++st) mt = fmaxf(mt, sc[st][g]);
+      if (mt > m[g] + DEC_TAU) {                  // false while both are -inf
+        const float a = ex2_approx(m[g] - mt);
+        l[g] *= a;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[g][e] *= a;
+        m[g] = mt;
+      }
+    }
+#pragma unroll
+    for (int st = 0; st < KS; ++st) {
+      const int kt = warp * (T / NW) + st * KPW + kg;
+      if (!full_tile && key0 + kt >= k_end) continue;   // never read V rows past the chunk end
+      float vf[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + kt * D * 2 + ds * 16), vf);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pr = ex2_approx(sc[st][g] - m[g]);
+        l[g] += pr;
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1], acc[g][e], acc[g][e + 1]);
       }
     }
     __syncwarp();
@@ -188,7 +238,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       const float c = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mn);
       l[g] = l[g] * a + lo * c;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
+      for (int e = 0; e < 8; ++e) {
         const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], o);
         acc[g][e] = acc[g][e] * a + ao * c;
       }
@@ -202,10 +252,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       float* dst = mrg + (warp * GP + g) * (D + 2);
       if (ds == 0) { dst[0] = m[g]; dst[1] = l[g]; }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        dst[2 + ds * 8 + e] = acc[g][e];
-        dst[2 + (ds + LPK) * 8 + e] = acc[g][8 + e];
-      }
+      for (int e = 0; e < 8; ++e) dst[2 + ds * 8 + e] = acc[g][e];
     }
   }
   asm volatile("bar.sync 1, %0;" :: "r"(NW * 32) : "memory");
