@@ -147,6 +147,7 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                      const fa::BwdParams& p, unsigned grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
+  if (!launch_regs_match(fa::bwd_main_kernel<D, CAUSAL>, fa::BWD_LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(fa::bwd_main_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
   fa::bwd_main_kernel<D, CAUSAL><<<grid, fa::BwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, mdo, p);
   return launch_status();

@@ -9,20 +9,23 @@
 // Three launches on the caller's stream (plus a memset of the dQ accumulator):
 //   bwd_pre_kernel   Delta, the LSE in log2 units (+inf for rows without a key,
 //                    so that their P is 0), both padded to 128-row tiles.
-//   bwd_main_kernel  one CTA per (batch, kv head, 128-key tile); loops over the
+//   bwd_main_kernel  one CTA per (batch, kv head, 128-key tile), head-major; loops over the
 //                    (query tile, query head of the group) pairs:
-//        warp 8     TMA: K, V once; Q, dO, LSE, Delta per pair (NQ stages)
-//        warp 9     tcgen05: S^T = K Q^T and dP^T = V dO^T into TMEM,
+//        warp 12    TMA: K, V once; Q, dO, LSE, Delta per pair (NQ stages)
+//        warp 13    tcgen05: S^T = K Q^T and dP^T = V dO^T into TMEM,
 //                   dV += P^T dO, dK += dS^T Q, dQ = dS K
 //        P^T and dS^T enter the products as bf16.  P^T = P_hi + P_lo and
 //        dS^T = dS_hi + dS_lo (each part bf16; P_hi in TMEM over S^T, the rest
 //        in swizzled shared memory); dV and dK take both parts, so that their
 //        only rounding is the fp32 accumulation, and dQ takes dS_hi.
-//        warps 0-3  one thread per key row: P^T from S^T and the LSE (causal /
-//                   ragged mask), P^T -> TMEM; dS^T = P^T (dP^T - Delta) -> smem
-//        warps 4-7  one thread per query row: dQ tile from TMEM added to the fp32
-//                   accumulator with vector atomics; at the end dK, dV out of TMEM
-//        warp 10    TMEM allocation
+//        warps 0-7  one thread per key row; warps w and w + 4 share a TMEM lane
+//                   quadrant and take 64 of the 128 query columns each (no row
+//                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
+//        warps 8-11 one thread per query row: dQ tile from TMEM (two buffers at
+//                   D = 64) added to the fp32 accumulator with vector atomics;
+//                   at the end dK, dV out of TMEM
+//        warp 14    TMEM allocation; warp 15 idles.  The control warpgroup
+//                   (12-15) lends registers to the other three.
 //   bwd_post_kernel  dQ = scale * accumulator, converted to the output dtype.
 #pragma once
 #include "sm100.cuh"
@@ -36,6 +39,7 @@ struct BwdCfg {
   static constexpr int NQ = (D == 64) ? 2 : 1;        // Q/dO stages (two do not fit at D = 128)
   static constexpr int NDS = 1;                       // one set of P_lo / dS_hi / dS_lo buffers
   static constexpr bool DQ_IN_DP = (D == 128);        // dQ reuses the dP^T columns
+  static constexpr int DQ_BUFS = DQ_IN_DP ? 1 : 2;    // dQ TMEM buffers
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = TILE;
   static constexpr int Q_OFF = 2 * TILE;              // stage s: Q at +s*2*TILE, dO after it
@@ -45,12 +49,12 @@ struct BwdCfg {
   static constexpr int PLO_OFF = DSLO_OFF + DS_BYTES; // low bf16 part of P^T
   static constexpr int ROW_OFF = PLO_OFF + DS_BYTES;  // stage s: lse2[128], delta[128]
   static constexpr int BAR_OFF = ROW_OFF + NQ * 1024;
-  static constexpr int NBARS = 1 + 2 * NQ + 3 + NDS + 4;
+  static constexpr int NBARS = 1 + 2 * NQ + 4 + 4 + 2;
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
-  static constexpr uint32_t T_DQ = DQ_IN_DP ? T_DP : 256 + 2 * D;
-  static constexpr int THREADS = 384;
+  static constexpr uint32_t T_DQ = DQ_IN_DP ? T_DP : 256 + 2 * D;   // buffer b at T_DQ + b * D
+  static constexpr int THREADS = 512;
 };
 
 struct BwdParams {
@@ -64,6 +68,9 @@ struct BwdParams {
   int g_fp32;
   uint64_t wait_limit_ns;
 };
+
+constexpr int BWD_LAUNCH_REGS = 128, BWD_WORK_REGS = 152, BWD_CTRL_REGS = 56;
+static_assert(3 * BWD_WORK_REGS + BWD_CTRL_REGS == 4 * BWD_LAUNCH_REGS, "register split must match the launch");
 
 enum : uint32_t {
   W_BWD_KV = 0x301, W_BWD_QF = 0x302, W_BWD_QE = 0x303, W_BWD_SDP = 0x304, W_BWD_P = 0x305,
@@ -127,12 +134,12 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* acc, void* d
 }
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int NQ = C::NQ, KB = D / 64;
+  constexpr int NQ = C::NQ, KB = D / 64, NB = C::DQ_BUFS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -143,19 +150,23 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* p_ready = sdp_full + 1;
   uint64_t* ds_ready = p_ready + 1;
   uint64_t* ds_free = ds_ready + 1;
-  uint64_t* dq_full = ds_free + 1;
-  uint64_t* dq_free = dq_full + 1;
-  uint64_t* dkv_done = dq_free + 1;
+  uint64_t* dq_full = ds_free + 1;       // [2]
+  uint64_t* dq_free = dq_full + 2;       // [2]
+  uint64_t* dkv_done = dq_free + 2;
   uint64_t* mma_done = dkv_done + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.wait_limit_ns;
   const int G = p.Hq / p.Hkv;
-  const int bk = p.B * p.Hkv;
-  const int j = static_cast<int>(blockIdx.x / bk);        // key tile, heaviest (j = 0) first
-  const int b = static_cast<int>(blockIdx.x % bk) / p.Hkv;
-  const int hkv = static_cast<int>(blockIdx.x % bk) % p.Hkv;
+  // Head-major order: the key tiles of one (b, kv head) are adjacent (heaviest,
+  // j = 0, first), so the CTAs running at the same time touch a few heads' Q,
+  // dO and fp32 dQ accumulator, which then stay in L2 (all heads together do not).
+  const int nk = (p.Lk + 127) >> 7;
+  const int j = static_cast<int>(blockIdx.x % nk);
+  const int bh = static_cast<int>(blockIdx.x / nk);
+  const int b = bh / p.Hkv;
+  const int hkv = bh % p.Hkv;
   const int off = p.Lk - p.Lq;
   const int nq = (p.Lq + 127) >> 7;
   int i0 = 0;
@@ -169,22 +180,23 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(kv_full, 1);
     for (int s = 0; s < NQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     mbar_init(sdp_full, 1);
-    mbar_init(p_ready, 128);
-    mbar_init(ds_ready, 128);
+    mbar_init(p_ready, 256);
+    mbar_init(ds_ready, 256);
     mbar_init(ds_free, 1);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
+    for (int u = 0; u < 2; ++u) { mbar_init(&dq_full[u], 1); mbar_init(&dq_free[u], 128); }
     mbar_init(dkv_done, 1);
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == 10) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  if (warp == 14) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 8) {
+  if (warp >= 12) {
+  setmaxnreg_dec<BWD_CTRL_REGS>();
+  if (warp == 12) {
     // ------------------------------------------------------------ producer --
     if (lane == 0 && npairs > 0) {
       tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_do);
@@ -213,7 +225,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_wait(kv_full, 0, lim, W_BWD_DRAIN);
       for (int n = max(0, issued - NQ); n < issued; ++n) mbar_wait(&q_full[n % NQ], (n / NQ) & 1, lim, W_BWD_DRAIN);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0 && npairs > 0) {
       constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
@@ -235,21 +247,21 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_after();
       if (ok) { issue_s_dp(0); umma_commit(sdp_full); }
       for (int n = 0; ok && n < npairs; ++n) {
-        const int s = n % NQ;
+        const int s = n % NQ, bq = n % NB;
         const uint32_t qa = q_base + s * 2 * C::TILE, da = qa + C::TILE;
-        const uint32_t dsa = ds_base;
         if (!(ok = mbar_wait(p_ready, n & 1, lim, W_BWD_P))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // dV += P_hi^T dO  (K = 128 queries)
-          umma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)      // dV += P_hi^T dO  (K = 128 queries; P_hi of query
+          umma_ts(tmem + C::T_DV,           // columns [64h, 64h+64) sits in TMEM columns [64h, 64h+32))
+                  tmem + C::T_S + (kk >> 2) * 64 + (kk & 3) * 8, mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
         if (!(ok = mbar_wait(ds_ready, n & 1, lim, W_BWD_DS))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dV += P_lo^T dO
           umma_ss(tmem + C::T_DV, kmaj(plo_base, kk), mnmaj(da, kk), ID_DVK, 1u);
         const bool more = n + 1 < npairs;
-        if (!C::DQ_IN_DP && more) {         // next pair's S^T, dP^T first: the softmax warps start early
+        if (!C::DQ_IN_DP && more) {         // next pair's S^T, dP^T first: the compute warps start early
           if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
           tc_fence_after();
           issue_s_dp(n + 1);
@@ -257,22 +269,22 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dK += dS_hi^T Q  (K = 128 queries)
-          umma_ss(tmem + C::T_DK, kmaj(dsa, kk), mnmaj(qa, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
+          umma_ss(tmem + C::T_DK, kmaj(ds_base, kk), mnmaj(qa, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dK += dS_lo^T Q
           umma_ss(tmem + C::T_DK, kmaj(dslo_base, kk), mnmaj(qa, kk), ID_DVK, 1u);
-        if (!C::DQ_IN_DP && n > 0) {        // dQ(n-1) must have been read out of TMEM
-          if (!(ok = mbar_wait(dq_free, (n - 1) & 1, lim, W_BWD_DQF))) break;
+        if (!C::DQ_IN_DP && n >= NB) {      // this dQ buffer must have been read out (pair n - NB)
+          if (!(ok = mbar_wait(&dq_free[bq], ((n / NB) - 1) & 1, lim, W_BWD_DQF))) break;
           tc_fence_after();
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dQ = dS K  (K = 128 keys)
-          umma_ss(tmem + C::T_DQ, mnmaj(dsa, kk), mnmaj(k_base, kk), ID_DQ, kk > 0 ? 1u : 0u);
-        umma_commit(dq_full);
+          umma_ss(tmem + C::T_DQ + bq * D, mnmaj(ds_base, kk), mnmaj(k_base, kk), ID_DQ, kk > 0 ? 1u : 0u);
+        umma_commit(&dq_full[bq]);
         umma_commit(ds_free);
         umma_commit(&q_empty[s]);
         if (C::DQ_IN_DP && more) {          // dP^T(n+1) overwrites dQ(n): wait for its read-out
-          if (!(ok = mbar_wait(dq_free, n & 1, lim, W_BWD_DQF))) break;
+          if (!(ok = mbar_wait(&dq_free[0], n & 1, lim, W_BWD_DQF))) break;
           if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
           tc_fence_after();
           issue_s_dp(n + 1);
@@ -283,12 +295,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, lim, W_BWD_DONE);
     }
-  } else if (warp < 4) {
+  }
+  // take the launch budget back only after the other warpgroups returned theirs
+  asm volatile("bar.sync 2, %0;" :: "n"(C::THREADS) : "memory");
+  setmaxnreg_inc<BWD_LAUNCH_REGS>();
+  } else if (warp < 8) {
+    setmaxnreg_inc<BWD_WORK_REGS>();
     // --------------------------------------------- P^T and dS^T (key rows) --
-    const int r = warp * 32 + lane;
+    const int wq = warp & 3, hh = warp >> 2;          // lane quadrant, which 64 query columns
+    const int r = wq * 32 + lane;
     const int key = j * 128 + r;
-    const bool key_ok = key < p.Lk;
-    const uint32_t lane_bits = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const float sl2 = p.scale_log2;
     for (int n = 0; n < npairs; ++n) {
       const int s = n % NQ;
@@ -297,43 +314,48 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float* dlt = lse2 + 128;
       if (!mbar_wait_warp(sdp_full, n & 1, lim, W_BWD_SDP)) break;
       tc_fence_after();
-      // allowed when key <= query + off, i.e. column c >= cmin
-      const int cmin = CAUSAL ? key - off - i * 128 : -1;
+      // allowed when key <= query + off, i.e. column c >= cmin (nothing for keys past Lk)
+      const int cmin = key < p.Lk ? (CAUSAL ? key - off - i * 128 : -1) : (1 << 30);
       const int rowoff = r * 128;
       bool ok = true;
-      // 32 query columns per step.  P_hi (bf16) of columns [32ch, 32ch+32) goes to
-      // TMEM columns [16ch, 16ch+16) of the S^T block, below every S^T column
-      // still to be read; P_lo, dS_hi and dS_lo go to shared memory.
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int lc = 0; lc < 2; ++lc) {
+        const int c0 = hh * 64 + lc * 32;              // first query column of this chunk
         uint32_t sv[32], dp[32];
-        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_S + ch * 32, sv);
-        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DP + ch * 32, dp);
+        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_S + c0, sv);
+        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DP + c0, dp);
         uint32_t phi[16], plo[16], dhi[16], dlo[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-          const int c = ch * 32 + 2 * t;
+          const int c = c0 + 2 * t;
           const float2 l2 = *reinterpret_cast<const float2*>(lse2 + c);
           const float2 d2 = *reinterpret_cast<const float2*>(dlt + c);
-          float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * t]), sl2, -l2.x));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * t + 1]), sl2, -l2.y));
-          p0 = (key_ok && c >= cmin) ? p0 : 0.f;
-          p1 = (key_ok && c + 1 >= cmin) ? p1 : 0.f;
+          float x0, x1;
+          ffma2(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), sl2, sl2, -l2.x, -l2.y);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          p0 = (c >= cmin) ? p0 : 0.f;
+          p1 = (c + 1 >= cmin) ? p1 : 0.f;
           phi[t] = pack_bf16x2(p0, p1);
-          plo[t] = pack_bf16x2(p0 - __uint_as_float(phi[t] << 16), p1 - __uint_as_float(phi[t] & 0xffff0000u));
-          const float s0 = p0 * (__uint_as_float(dp[2 * t]) - d2.x);
-          const float s1 = p1 * (__uint_as_float(dp[2 * t + 1]) - d2.y);
+          float r0, r1;
+          fadd2(r0, r1, p0, p1, -__uint_as_float(phi[t] << 16), -__uint_as_float(phi[t] & 0xffff0000u));
+          plo[t] = pack_bf16x2(r0, r1);
+          float e0, e1, s0, s1;
+          fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -d2.x, -d2.y);
+          ffma2(s0, s1, p0, p1, e0, e1, 0.f, 0.f);
           dhi[t] = pack_bf16x2(s0, s1);
-          dlo[t] = pack_bf16x2(s0 - __uint_as_float(dhi[t] << 16), s1 - __uint_as_float(dhi[t] & 0xffff0000u));
+          fadd2(r0, r1, s0, s1, -__uint_as_float(dhi[t] << 16), -__uint_as_float(dhi[t] & 0xffff0000u));
+          dlo[t] = pack_bf16x2(r0, r1);
         }
-        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + ch * 16, phi);
+        // P_hi of columns [c0, c0+32) -> TMEM columns hh*64 + lc*16 .. +16: inside this
+        // warp's own S columns, all of which it has already read
+        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + hh * 64 + lc * 16, phi);
         // the shared-memory operands of pair n - 1 must have been consumed
-        if (ch == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
-        // 32 columns = 4 16-byte chunks of the 128-byte row of block ch/2 (128B swizzle)
-        const int blk = (ch >> 1) * 16384 + rowoff;
+        if (lc == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
+        // columns c0..c0+31: 4 16-byte chunks of the 128-byte row of block hh (128B swizzle)
+        const int blk = hh * 16384 + rowoff;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int o16 = blk + ((((ch & 1) * 4 + t) ^ (r & 7)) << 4);
+          const int o16 = blk + (((lc * 4 + t) ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(smem + C::PLO_OFF + o16) = make_uint4(plo[4 * t], plo[4 * t + 1], plo[4 * t + 2], plo[4 * t + 3]);
           *reinterpret_cast<uint4*>(smem + C::DS_OFF + o16) = make_uint4(dhi[4 * t], dhi[4 * t + 1], dhi[4 * t + 2], dhi[4 * t + 3]);
           *reinterpret_cast<uint4*>(smem + C::DSLO_OFF + o16) = make_uint4(dlo[4 * t], dlo[4 * t + 1], dlo[4 * t + 2], dlo[4 * t + 3]);
@@ -346,14 +368,18 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_arrive(p_ready);
       mbar_arrive(ds_ready);
     }
-  } else if (warp < 8) {
+    setmaxnreg_dec<BWD_LAUNCH_REGS>();
+    asm volatile("bar.arrive 2, %0;" :: "n"(C::THREADS) : "memory");
+  } else {
+    setmaxnreg_inc<BWD_WORK_REGS>();
     // ------------------------------------- dQ read-out, then dK/dV epilogue --
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     bool ok = true;
     for (int n = 0; n < npairs; ++n) {
-      if (!(ok = mbar_wait_warp(dq_full, n & 1, lim, W_BWD_DQ))) break;
+      const int bq = n % NB;
+      if (!(ok = mbar_wait_warp(&dq_full[bq], (n / NB) & 1, lim, W_BWD_DQ))) break;
       tc_fence_after();
       const int i = i0 + n / G, hq = hkv * G + n % G;
       const int qrow = i * 128 + r;
@@ -361,7 +387,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DQ + c0, v);
+        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DQ + bq * D + c0, v);
         if (qrow < p.Lq) {
 #pragma unroll
           for (int t = 0; t < 8; ++t)
@@ -371,7 +397,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       tc_fence_before();
-      mbar_arrive(dq_free);
+      mbar_arrive(&dq_free[bq]);
     }
     const bool have = ok && npairs > 0 && mbar_wait_warp(dkv_done, 0, lim, W_BWD_DKV);
     if (have) tc_fence_after();
@@ -408,11 +434,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
     }
+    setmaxnreg_dec<BWD_LAUNCH_REGS>();
+    asm volatile("bar.arrive 2, %0;" :: "n"(C::THREADS) : "memory");
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 10) {
+  if (warp == 14) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
