@@ -69,7 +69,7 @@ struct BwdParams {
   uint64_t wait_limit_ns;
 };
 
-constexpr int BWD_LAUNCH_REGS = 128, BWD_WORK_REGS = 152, BWD_CTRL_REGS = 56;
+constexpr int BWD_LAUNCH_REGS = 128, BWD_WORK_REGS = 136, BWD_CTRL_REGS = 104;
 static_assert(3 * BWD_WORK_REGS + BWD_CTRL_REGS == 4 * BWD_LAUNCH_REGS, "register split must match the launch");
 
 enum : uint32_t {
