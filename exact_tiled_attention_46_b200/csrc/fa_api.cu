@@ -77,6 +77,18 @@ bool ensure_smem_attr(F* func, int bytes, std::atomic<uint64_t>& done_mask) {
 
 fa_status launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
+// Number of SMs of the current device (cached per device); 0 on failure.
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 __global__ void fill_empty_rows_kernel(void* o, float* lse, size_t n_o, size_t n_lse, int o_fp32) {
   const size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x;
   const size_t stride = size_t(gridDim.x) * blockDim.x;
@@ -191,8 +203,8 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
   if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return FA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
   const long long pairs = (static_cast<long long>(Lq) + 255) / 256;
-  const long long grid = pairs * B * Hq;
-  if (!fits_int(grid) || !fits_int(static_cast<long long>(B) * Hq)) return FA_ERR_UNSUPPORTED;
+  const long long items = pairs * B * Hq;          // work items of the persistent grid
+  if (!fits_int(items) || !fits_int(static_cast<long long>(B) * Hq)) return FA_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (Lq == 0) return FA_OK;
   if (Lk == 0) {
@@ -210,6 +222,9 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_fp32 = (o_dtype == FA_FP32);
   p.wait_limit_ns = g_wait_limit_ns.load();
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long grid = items < sms ? items : sms;
   if (D == 128) return causal ? launch_fwd<128, true>(mq, mk, mv, p, grid, st) : launch_fwd<128, false>(mq, mk, mv, p, grid, st);
   return causal ? launch_fwd<64, true>(mq, mk, mv, p, grid, st) : launch_fwd<64, false>(mq, mk, mv, p, grid, st);
 }

@@ -3,11 +3,15 @@
 // and Use Less Memory", sections "1. Tiling", "3. Online Softmax" and "Fused
 // Computation"; "Flash Attention Explained: Same Maths, Far Less Memory",
 // section "The idea: never materialise the matrix").  The score matrix lives
-// only in tensor memory; HBM sees Q, K, V once per CTA and O/LSE once.
+// only in tensor memory; Q is read and O/LSE written once, K and V once per
+// work item (the re-reads of a head's K and V by its other items hit L2).
 //
-// One CTA owns two 128-row query tiles of one (batch, head) and walks the key
-// tiles of its kv head:
-//   warp 8      TMA producer: Q tiles once, then K_j, V_j into a slot ring
+// The grid is persistent (at most one CTA per SM).  A work item is a pair of
+// 128-row query tiles of one (batch, head); a CTA takes its items one after the
+// other and, for each, walks the key tiles of the kv head:
+//   warp 8      TMA producer: the item's Q tiles (each slot refilled once the
+//               previous item's last S on it is done), then K_j, V_j into a
+//               slot ring that runs on from item to item
 //   warp 9      MMA issuer:   S_t = Q_t K_j^T into TMEM, O_t += P_t V_j
 //   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: one
 //               thread per query row; causal / ragged mask; running max m and
@@ -19,7 +23,7 @@
 // SM sub-partition); the control warpgroup (warps 8-11) gives registers back
 // (setmaxnreg.dec to FWD_CTRL_REGS) and the two softmax warpgroups take them
 // (setmaxnreg.inc to FWD_SOFTMAX_REGS).  The split sums to exactly the launch
-// allocation: 2 * 224 + 56 = 3 * 168 registers per lane slot.
+// allocation: 2 * 208 + 88 = 3 * 168 registers per lane slot.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 #pragma once
 #include "sm100.cuh"
@@ -44,7 +48,7 @@ struct FwdCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
-  static constexpr int NBARS = 1 + 2 * NS + 2 + 2 + 2 + 1;
+  static constexpr int NBARS = 2 + 2 + 2 * NS + 2 + 2 + 2 + 1;
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
   static constexpr int THREADS = 384;
 };
@@ -57,7 +61,7 @@ struct FwdCfg {
 // when it grows by more than FWD_TAU, O and the sums are rescaled in place, and
 // P is recomputed.
 constexpr float FWD_TAU = 8.0f;
-constexpr int FWD_LAUNCH_REGS = 168, FWD_SOFTMAX_REGS = 224, FWD_CTRL_REGS = 56;
+constexpr int FWD_LAUNCH_REGS = 168, FWD_SOFTMAX_REGS = 208, FWD_CTRL_REGS = 88;
 static_assert(2 * FWD_SOFTMAX_REGS + FWD_CTRL_REGS == 3 * FWD_LAUNCH_REGS, "register split must match the launch");
 constexpr float FWD_FAST_LIMIT = 65536.0f;
 
@@ -84,8 +88,51 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
 
 enum : uint32_t {
   W_FWD_Q = 0x101, W_FWD_KV_EMPTY = 0x102, W_FWD_KV_FULL = 0x103, W_FWD_P = 0x104,
-  W_FWD_S = 0x105, W_FWD_O = 0x106, W_FWD_DONE = 0x107, W_FWD_DRAIN = 0x108
+  W_FWD_S = 0x105, W_FWD_O = 0x106, W_FWD_DONE = 0x107, W_FWD_DRAIN = 0x108, W_FWD_Q_EMPTY = 0x109
 };
+
+// One work item is a pair of 128-row query tiles of one (batch, head).  Items
+// are numbered heaviest first (causal work grows with the pair index); the grid
+// is persistent (at most one CTA per SM) and CTA c takes, in round r, item
+// r * G + c (r even) or r * G + G - 1 - c (r odd), a boustrophedon order that
+// evens out the causal work across CTAs.
+struct FwdItem {
+  int b, h, hkv, q0, n_t0, n_t1, n;
+};
+template <bool CAUSAL>
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
+  FwdItem I;
+  const int bh_count = p.B * p.Hq;
+  const int pair = p.num_pairs - 1 - w / bh_count;
+  const int bh = w % bh_count;
+  I.b = bh / p.Hq;
+  I.h = bh % p.Hq;
+  I.hkv = I.h / (p.Hq / p.Hkv);
+  I.q0 = pair * 256;
+  const int off = p.Lk - p.Lq;
+  const int nk_all = (p.Lk + 127) >> 7;
+  int nt[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = I.q0 + t * 128;
+    if (r0 >= p.Lq) {
+      nt[t] = 0;
+    } else if (!CAUSAL) {
+      nt[t] = nk_all;
+    } else {
+      const int lim_keys = min(r0 + 127, p.Lq - 1) + off + 1;   // keys < lim_keys for the last row
+      nt[t] = lim_keys <= 0 ? 0 : min(nk_all, (lim_keys + 127) >> 7);
+    }
+  }
+  I.n_t0 = nt[0];
+  I.n_t1 = nt[1];
+  I.n = max(nt[0], nt[1]);
+  return I;
+}
+__device__ __forceinline__ int fwd_item_index(int r) {
+  const int G = static_cast<int>(gridDim.x);
+  return r * G + ((r & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x));
+}
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
@@ -97,47 +144,28 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-  uint64_t* bar_q = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
+  uint64_t* q_full = bars;                         // [2] Q tile t landed
+  uint64_t* q_empty = q_full + 2;                  // [2] last S of Q tile t done
+  uint64_t* kv_full = q_empty + 2;                 // [NS]
+  uint64_t* kv_empty = kv_full + NS;               // [NS]
+  uint64_t* s_full = kv_empty + NS;                // [2]
+  uint64_t* p_full = s_full + 2;                   // [2]
+  uint64_t* o_full = p_full + 2;                   // [2]
   uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.wait_limit_ns;
-
-  // heaviest query-tile pairs first (causal work grows with the pair index)
-  const int bh_count = p.B * p.Hq;
-  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x / bh_count);
-  const int bh = static_cast<int>(blockIdx.x % bh_count);
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int hkv = h / (p.Hq / p.Hkv);
-  const int q0 = pair * 256;
+  const int G = static_cast<int>(gridDim.x);
+  const int num_items = p.num_pairs * p.B * p.Hq;
   const int off = p.Lk - p.Lq;                     // bottom-right causal alignment
-  const int nk_all = (p.Lk + 127) >> 7;
-
-  int n_t[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int r0 = q0 + t * 128;
-    if (r0 >= p.Lq) {
-      n_t[t] = 0;
-    } else if (!CAUSAL) {
-      n_t[t] = nk_all;
-    } else {
-      const int lim_keys = min(r0 + 127, p.Lq - 1) + off + 1;   // keys < lim_keys for the last row
-      n_t[t] = lim_keys <= 0 ? 0 : min(nk_all, (lim_keys + 127) >> 7);
-    }
-  }
-  const int n = max(n_t[0], n_t[1]);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1); mbar_init(&q_empty[t], 1);
+      mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_full[t], 1);
+    }
     for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
-    for (int t = 0; t < 2; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_full[t], 1); }
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
@@ -152,29 +180,42 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   setmaxnreg_dec<FWD_CTRL_REGS>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
-      for (int t = 0; t < 2; ++t)
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(smem + C::Q_OFF + t * C::TILE_BYTES + kb * 16384, &tm_q, bar_q, kb * 64, h, q0 + t * 128, b);
-      int issued = 0;
-      for (int it = 0; it < 2 * n; ++it) {
-        const int slot = it % NS;
-        if (it >= NS && !mbar_wait(&kv_empty[slot], ((it / NS) + 1) & 1, lim, W_FWD_KV_EMPTY)) break;
-        mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
-        const CUtensorMap* m = (it & 1) ? &tm_v : &tm_k;
-        uint8_t* dst = smem + C::KV_OFF + slot * C::TILE_BYTES;
-        for (int kb = 0; kb < KB; ++kb) tma_load_4d(dst + kb * 16384, m, &kv_full[slot], kb * 64, hkv, (it >> 1) * 128, b);
-        issued = it + 1;
+    if (lane == 0) {
+      int it = 0;                                  // K/V ring loads issued
+      int q_cnt[2] = {0, 0};                       // Q loads issued per tile slot
+      bool ok = true;
+      for (int r = 0; ok && r * G < num_items; ++r) {
+        const int w = fwd_item_index(r);
+        if (w >= num_items) continue;
+        const FwdItem I = fwd_item<CAUSAL>(p, w);
+        if (I.n == 0) continue;
+        for (int t = 0; t < 2; ++t) {
+          if ((t ? I.n_t1 : I.n_t0) == 0) continue;
+          if (q_cnt[t] > 0 && !(ok = mbar_wait(&q_empty[t], (q_cnt[t] - 1) & 1, lim, W_FWD_Q_EMPTY))) break;
+          mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_4d(smem + C::Q_OFF + t * C::TILE_BYTES + kb * 16384, &tm_q, &q_full[t], kb * 64, I.h,
+                        I.q0 + t * 128, I.b);
+          ++q_cnt[t];
+        }
+        for (int i = 0; ok && i < 2 * I.n; ++i) {
+          const int slot = it % NS;
+          if (it >= NS && !(ok = mbar_wait(&kv_empty[slot], ((it / NS) + 1) & 1, lim, W_FWD_KV_EMPTY))) break;
+          mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
+          const CUtensorMap* m = (i & 1) ? &tm_v : &tm_k;
+          uint8_t* dst = smem + C::KV_OFF + slot * C::TILE_BYTES;
+          for (int kb = 0; kb < KB; ++kb) tma_load_4d(dst + kb * 16384, m, &kv_full[slot], kb * 64, I.hkv, (i >> 1) * 128, I.b);
+          ++it;
+        }
       }
       // the CTA may not exit with copies in flight: wait for the last loads
-      mbar_wait(bar_q, 0, lim, W_FWD_DRAIN);
-      for (int it = max(0, issued - NS); it < issued; ++it)
-        mbar_wait(&kv_full[it % NS], (it / NS) & 1, lim, W_FWD_DRAIN);
+      for (int t = 0; t < 2; ++t)
+        if (q_cnt[t] > 0) mbar_wait(&q_full[t], (q_cnt[t] - 1) & 1, lim, W_FWD_DRAIN);
+      for (int i = max(0, it - NS); i < it; ++i) mbar_wait(&kv_full[i % NS], (i / NS) & 1, lim, W_FWD_DRAIN);
     }
   } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
       const uint32_t q_base = smem_u32(smem + C::Q_OFF);
@@ -194,40 +235,59 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           umma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), IDESC_O,
                   (acc || kk > 0) ? 1u : 0u);
       };
-      auto wait_item = [&](int it) { return mbar_wait(&kv_full[it % NS], (it / NS) & 1, lim, W_FWD_KV_FULL); };
+      auto wait_item = [&](int i) { return mbar_wait(&kv_full[i % NS], (i / NS) & 1, lim, W_FWD_KV_FULL); };
 
-      bool ok = mbar_wait(bar_q, 0, lim, W_FWD_Q) && wait_item(0);
-      tc_fence_after();
-      if (ok) {
-        for (int t = 0; t < 2; ++t)
-          if (n_t[t] > 0) { issue_s(t, 0); umma_commit(&s_full[t]); }
-        umma_commit(&kv_empty[0]);
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        const int it_v = 2 * j + 1, it_k = 2 * j + 2;
-        if (!(ok = wait_item(it_v))) break;
-        tc_fence_after();
-        bool k_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= n_t[t]) continue;
-          if (!(ok = mbar_wait(&p_full[t], j & 1, lim, W_FWD_P))) break;
+      int it = 0;                                  // K/V ring loads consumed
+      int q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      bool ok = true;
+      for (int r = 0; ok && r * G < num_items; ++r) {
+        const int w = fwd_item_index(r);
+        if (w >= num_items) continue;
+        const FwdItem I = fwd_item<CAUSAL>(p, w);
+        if (I.n == 0) continue;
+        const int nt[2] = {I.n_t0, I.n_t1};
+        const int it0 = it;                        // K_j at it0 + 2j, V_j at it0 + 2j + 1
+        if (!(ok = wait_item(it0))) break;
+        for (int t = 0; t < 2; ++t) {
+          if (nt[t] == 0) continue;
+          if (!(ok = mbar_wait(&q_full[t], q_cnt[t] & 1, lim, W_FWD_Q))) break;
+          ++q_cnt[t];
           tc_fence_after();
-          issue_pv(t, it_v % NS, j > 0);
-          if (j + 1 < n_t[t]) {
-            if (!k_ready) {
-              if (!(ok = wait_item(it_k))) break;
-              tc_fence_after();
-              k_ready = true;
-            }
-            issue_s(t, it_k % NS);
-            umma_commit(&s_full[t]);
-          } else {
-            umma_commit(&o_full[t]);
-          }
+          issue_s(t, it0 % NS);
+          umma_commit(&s_full[t]);
+          if (nt[t] == 1) umma_commit(&q_empty[t]);
         }
         if (!ok) break;
-        umma_commit(&kv_empty[it_v % NS]);
-        if (k_ready) umma_commit(&kv_empty[it_k % NS]);
+        umma_commit(&kv_empty[it0 % NS]);
+        for (int j = 0; ok && j < I.n; ++j) {
+          const int it_v = it0 + 2 * j + 1, it_k = it0 + 2 * j + 2;
+          if (!(ok = wait_item(it_v))) break;
+          tc_fence_after();
+          bool k_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j >= nt[t]) continue;
+            if (!(ok = mbar_wait(&p_full[t], p_cnt[t] & 1, lim, W_FWD_P))) break;
+            ++p_cnt[t];
+            tc_fence_after();
+            issue_pv(t, it_v % NS, j > 0);
+            if (j + 1 < nt[t]) {
+              if (!k_ready) {
+                if (!(ok = wait_item(it_k))) break;
+                tc_fence_after();
+                k_ready = true;
+              }
+              issue_s(t, it_k % NS);
+              umma_commit(&s_full[t]);
+              if (j + 2 == nt[t]) umma_commit(&q_empty[t]);   // the last S of this Q tile
+            } else {
+              umma_commit(&o_full[t]);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&kv_empty[it_v % NS]);
+          if (k_ready) umma_commit(&kv_empty[it_k % NS]);
+        }
+        it = it0 + 2 * I.n;
       }
       // nothing may be in flight on the tensor pipe when the CTA tears down
       umma_commit(mma_done);
@@ -244,130 +304,139 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     // ------------------------------------------------------------- softmax --
     const int t = warp >> 2;
     const int wq = warp & 3;                       // TMEM lane quadrant of this warp
-    const int row = q0 + t * 128 + wq * 32 + lane; // global query row of this thread
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_bits + t * 128;
     const uint32_t t_o = tmem + lane_bits + 256 + t * D;
-    const int nt = n_t[t];
     const float sl2 = p.scale_log2;
-    const int row_tile0 = q0 + t * 128;
-    // l: exact fp32 sum of p (for LSE); lr: sum of the bf16-rounded p that the
-    // P.V product uses (the normaliser of O)
-    float m_used = -INFINITY, l = 0.f, lr = 0.f;
+    int s_cnt = 0, o_cnt = 0;                      // phases consumed on s_full[t], o_full[t]
     bool ok = true;
+    for (int r = 0; ok && r * G < num_items; ++r) {
+      const int w = fwd_item_index(r);
+      if (w >= num_items) continue;
+      const FwdItem I = fwd_item<CAUSAL>(p, w);
+      const int b = I.b, h = I.h;
+      const int row_tile0 = I.q0 + t * 128;
+      const int row = row_tile0 + wq * 32 + lane;    // global query row of this thread
+      const int nt = t ? I.n_t1 : I.n_t0;
+      // l: exact fp32 sum of p (for LSE); lr: sum of the bf16-rounded p that the
+      // P.V product uses (the normaliser of O)
+      float m_used = -INFINITY, l = 0.f, lr = 0.f;
 
-    for (int j = 0; j < nt; ++j) {
-      if (!(ok = mbar_wait_warp(&s_full[t], j & 1, lim, W_FWD_S))) break;
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld_32x32b_x128(t_s, sr);
-      float* s = reinterpret_cast<float*>(sr);
-      const int kbase = j * 128;
-      const bool need_mask = (kbase + 128 > p.Lk) || (CAUSAL && kbase + 127 > row_tile0 + off);
-      if (need_mask) {
-        int lim_c = p.Lk - kbase;
-        if (CAUSAL) lim_c = min(lim_c, row + off + 1 - kbase);
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = (c < lim_c) ? s[c] : -INFINITY;
-      }
-      float ls0 = 0.f, ls1 = 0.f, lr0 = 0.f, lr1 = 0.f;
-      // P = 2^(s*scale*log2e - m), packed to bf16 and stored over the first 64
-      // columns of S; ls = exact sum, lr = sum of the bf16 values (O's normaliser)
-      auto exp_tile = [&](float msub, bool use_poly) {
-        ls0 = ls1 = lr0 = lr1 = 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = half * 64 + 2 * i;
-            float x0, x1, p0, p1;
-            ffma2(x0, x1, s[c], s[c + 1], sl2, sl2, -msub, -msub);
-            if (use_poly && (i % 3) == 2) {
-              exp2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+      for (int j = 0; j < nt; ++j) {
+        if (!(ok = mbar_wait_warp(&s_full[t], s_cnt & 1, lim, W_FWD_S))) break;
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld_32x32b_x128(t_s, sr);
+        float* s = reinterpret_cast<float*>(sr);
+        const int kbase = j * 128;
+        const bool need_mask = (kbase + 128 > p.Lk) || (CAUSAL && kbase + 127 > row_tile0 + off);
+        if (need_mask) {
+          int lim_c = p.Lk - kbase;
+          if (CAUSAL) lim_c = min(lim_c, row + off + 1 - kbase);
+  #pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = (c < lim_c) ? s[c] : -INFINITY;
+        }
+        float ls0 = 0.f, ls1 = 0.f, lr0 = 0.f, lr1 = 0.f;
+        // P = 2^(s*scale*log2e - m), packed to bf16 and stored over the first 64
+        // columns of S; ls = exact sum, lr = sum of the bf16 values (O's normaliser)
+        auto exp_tile = [&](float msub, bool use_poly) {
+          ls0 = ls1 = lr0 = lr1 = 0.f;
+  #pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int c = half * 64 + 2 * i;
+              float x0, x1, p0, p1;
+              ffma2(x0, x1, s[c], s[c + 1], sl2, sl2, -msub, -msub);
+              if (use_poly && (i % 3) == 2) {
+                exp2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              pk[i] = pack_bf16x2(p0, p1);
+              fadd2(ls0, ls1, ls0, ls1, p0, p1);
+              add_bf16x2_f32(lr0, lr1, pk[i]);
             }
-            pk[i] = pack_bf16x2(p0, p1);
-            fadd2(ls0, ls1, ls0, ls1, p0, p1);
-            add_bf16x2_f32(lr0, lr1, pk[i]);
+            tmem_st_32x32b_x32(t_s + half * 32, pk);
           }
-          tmem_st_32x32b_x32(t_s + half * 32, pk);
+        };
+        bool slow = __any_sync(0xffffffffu, m_used == -INFINITY);
+        if (!slow) {
+          // the branch keeps the polynomial loop and the all-MUFU loop apart, so
+          // that the compiler cannot evaluate both and select
+          if (need_mask) exp_tile(m_used, false);
+          else exp_tile(m_used, true);
+          slow = __any_sync(0xffffffffu, !(ls0 + ls1 <= FWD_FAST_LIMIT));
         }
-      };
-      bool slow = __any_sync(0xffffffffu, m_used == -INFINITY);
-      if (!slow) {
-        // the branch keeps the polynomial loop and the all-MUFU loop apart, so
-        // that the compiler cannot evaluate both and select
-        if (need_mask) exp_tile(m_used, false);
-        else exp_tile(m_used, true);
-        slow = __any_sync(0xffffffffu, !(ls0 + ls1 <= FWD_FAST_LIMIT));
-      }
-      if (slow) {
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]); mx2 = fmaxf(mx2, s[c + 2]); mx3 = fmaxf(mx3, s[c + 3]);
-        }
-        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-        const bool resc = m_tile > m_used + FWD_TAU;   // false while both are -inf
-        float alpha = 1.f;
-        if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; lr *= alpha; m_used = m_tile; }
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld_32x32b_x32(t_o + c0, ov);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st_32x32b_x32(t_o + c0, ov);
+        if (slow) {
+          float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+  #pragma unroll
+          for (int c = 4; c < 128; c += 4) {
+            mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]); mx2 = fmaxf(mx2, s[c + 2]); mx3 = fmaxf(mx3, s[c + 3]);
           }
+          const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+          const bool resc = m_tile > m_used + FWD_TAU;   // false while both are -inf
+          float alpha = 1.f;
+          if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; lr *= alpha; m_used = m_tile; }
+          if (j > 0 && __any_sync(0xffffffffu, resc)) {
+  #pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld_32x32b_x32(t_o + c0, ov);
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st_32x32b_x32(t_o + c0, ov);
+            }
+          }
+          exp_tile((m_used == -INFINITY) ? 0.f : m_used, false);
         }
-        exp_tile((m_used == -INFINITY) ? 0.f : m_used, false);
+        l += ls0 + ls1;
+        lr += lr0 + lr1;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
       }
-      l += ls0 + ls1;
-      lr += lr0 + lr1;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
 
-    // ------------------------------------------------------------ epilogue --
-    const bool have_o = ok && nt > 0 && mbar_wait_warp(&o_full[t], 0, lim, W_FWD_O);
-    if (have_o) tc_fence_after();
-    const bool has = l > 0.f;
-    const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
-    const bool in_range = row < p.Lq;
-    if (in_range && p.lse != nullptr)
-      p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_used + log2f(l)) * LN2 : -INFINITY;
-    const size_t orow = (static_cast<size_t>(b) * p.Lq + row) * p.Hq + h;
-#pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t ov[32];
-      if (have_o) {
-        tmem_ld_32x32b_x32(t_o + c0, ov);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = 0u;
-      }
-      if (!in_range) continue;
-      if (p.o_fp32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
-                               __uint_as_float(ov[4 * i + 2]) * inv_l, __uint_as_float(ov[4 * i + 3]) * inv_l);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D + c0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]) * inv_l, __uint_as_float(ov[8 * i + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]) * inv_l, __uint_as_float(ov[8 * i + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]) * inv_l, __uint_as_float(ov[8 * i + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]) * inv_l, __uint_as_float(ov[8 * i + 7]) * inv_l);
-          dst[i] = w;
+      // ------------------------------------------------------------ epilogue --
+      const bool have_o = ok && nt > 0 && mbar_wait_warp(&o_full[t], o_cnt & 1, lim, W_FWD_O);
+      if (nt > 0) ++o_cnt;
+      if (have_o) tc_fence_after();
+      const bool has = l > 0.f;
+      const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
+      const bool in_range = row < p.Lq;
+      if (in_range && p.lse != nullptr)
+        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_used + log2f(l)) * LN2 : -INFINITY;
+      const size_t orow = (static_cast<size_t>(b) * p.Lq + row) * p.Hq + h;
+  #pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        if (have_o) {
+          tmem_ld_32x32b_x32(t_o + c0, ov);
+        } else {
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = 0u;
+        }
+        if (!in_range) continue;
+        if (p.o_fp32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c0);
+  #pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
+                                 __uint_as_float(ov[4 * i + 2]) * inv_l, __uint_as_float(ov[4 * i + 3]) * inv_l);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D + c0);
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 wv;
+            wv.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]) * inv_l, __uint_as_float(ov[8 * i + 1]) * inv_l);
+            wv.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]) * inv_l, __uint_as_float(ov[8 * i + 3]) * inv_l);
+            wv.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]) * inv_l, __uint_as_float(ov[8 * i + 5]) * inv_l);
+            wv.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]) * inv_l, __uint_as_float(ov[8 * i + 7]) * inv_l);
+            dst[i] = wv;
+          }
         }
       }
     }
