@@ -23,7 +23,7 @@
 // SM sub-partition); the control warpgroup (warps 8-11) gives registers back
 // (setmaxnreg.dec to FWD_CTRL_REGS) and the two softmax warpgroups take them
 // (setmaxnreg.inc to FWD_SOFTMAX_REGS).  The split sums to exactly the launch
-// allocation: 2 * 208 + 88 = 3 * 168 registers per lane slot.
+// allocation: 2 * 224 + 56 = 3 * 168 registers per lane slot.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 #pragma once
 #include "sm100.cuh"
@@ -61,7 +61,7 @@ struct FwdCfg {
 // when it grows by more than FWD_TAU, O and the sums are rescaled in place, and
 // P is recomputed.
 constexpr float FWD_TAU = 8.0f;
-constexpr int FWD_LAUNCH_REGS = 168, FWD_SOFTMAX_REGS = 208, FWD_CTRL_REGS = 88;
+constexpr int FWD_LAUNCH_REGS = 168, FWD_SOFTMAX_REGS = 224, FWD_CTRL_REGS = 56;
 static_assert(2 * FWD_SOFTMAX_REGS + FWD_CTRL_REGS == 3 * FWD_LAUNCH_REGS, "register split must match the launch");
 constexpr float FWD_FAST_LIMIT = 65536.0f;
 
@@ -182,21 +182,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       int it = 0;                                  // K/V ring loads issued
-      int q_cnt[2] = {0, 0};                       // Q loads issued per tile slot
+      uint32_t q_loaded = 0, q_par = 0;            // bit t: Q slot t loaded before / parity of its loads
       bool ok = true;
       for (int r = 0; ok && r * G < num_items; ++r) {
         const int w = fwd_item_index(r);
         if (w >= num_items) continue;
         const FwdItem I = fwd_item<CAUSAL>(p, w);
         if (I.n == 0) continue;
+#pragma unroll 1
         for (int t = 0; t < 2; ++t) {
           if ((t ? I.n_t1 : I.n_t0) == 0) continue;
-          if (q_cnt[t] > 0 && !(ok = mbar_wait(&q_empty[t], (q_cnt[t] - 1) & 1, lim, W_FWD_Q_EMPTY))) break;
+          // wait for the previous item's last S on this slot (phase = loads so far - 1)
+          if (((q_loaded >> t) & 1u) && !(ok = mbar_wait(&q_empty[t], ((q_par >> t) & 1u) ^ 1u, lim, W_FWD_Q_EMPTY))) break;
           mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
           for (int kb = 0; kb < KB; ++kb)
             tma_load_4d(smem + C::Q_OFF + t * C::TILE_BYTES + kb * 16384, &tm_q, &q_full[t], kb * 64, I.h,
                         I.q0 + t * 128, I.b);
-          ++q_cnt[t];
+          q_loaded |= 1u << t;
+          q_par ^= 1u << t;
         }
         for (int i = 0; ok && i < 2 * I.n; ++i) {
           const int slot = it % NS;
@@ -210,7 +213,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       }
       // the CTA may not exit with copies in flight: wait for the last loads
       for (int t = 0; t < 2; ++t)
-        if (q_cnt[t] > 0) mbar_wait(&q_full[t], (q_cnt[t] - 1) & 1, lim, W_FWD_DRAIN);
+        if ((q_loaded >> t) & 1u) mbar_wait(&q_full[t], ((q_par >> t) & 1u) ^ 1u, lim, W_FWD_DRAIN);
       for (int i = max(0, it - NS); i < it; ++i) mbar_wait(&kv_full[i % NS], (i / NS) & 1, lim, W_FWD_DRAIN);
     }
   } else if (warp == 9) {
@@ -238,24 +241,25 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       auto wait_item = [&](int i) { return mbar_wait(&kv_full[i % NS], (i / NS) & 1, lim, W_FWD_KV_FULL); };
 
       int it = 0;                                  // K/V ring loads consumed
-      int q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      uint32_t q_par = 0, p_par = 0;               // bit t: parity of the next q_full / p_full phase
       bool ok = true;
       for (int r = 0; ok && r * G < num_items; ++r) {
         const int w = fwd_item_index(r);
         if (w >= num_items) continue;
         const FwdItem I = fwd_item<CAUSAL>(p, w);
         if (I.n == 0) continue;
-        const int nt[2] = {I.n_t0, I.n_t1};
         const int it0 = it;                        // K_j at it0 + 2j, V_j at it0 + 2j + 1
         if (!(ok = wait_item(it0))) break;
+#pragma unroll 1
         for (int t = 0; t < 2; ++t) {
-          if (nt[t] == 0) continue;
-          if (!(ok = mbar_wait(&q_full[t], q_cnt[t] & 1, lim, W_FWD_Q))) break;
-          ++q_cnt[t];
+          const int ntt = t ? I.n_t1 : I.n_t0;
+          if (ntt == 0) continue;
+          if (!(ok = mbar_wait(&q_full[t], (q_par >> t) & 1u, lim, W_FWD_Q))) break;
+          q_par ^= 1u << t;
           tc_fence_after();
           issue_s(t, it0 % NS);
           umma_commit(&s_full[t]);
-          if (nt[t] == 1) umma_commit(&q_empty[t]);
+          if (ntt == 1) umma_commit(&q_empty[t]);
         }
         if (!ok) break;
         umma_commit(&kv_empty[it0 % NS]);
@@ -264,13 +268,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           if (!(ok = wait_item(it_v))) break;
           tc_fence_after();
           bool k_ready = false;
+#pragma unroll 1
           for (int t = 0; t < 2 && ok; ++t) {
-            if (j >= nt[t]) continue;
-            if (!(ok = mbar_wait(&p_full[t], p_cnt[t] & 1, lim, W_FWD_P))) break;
-            ++p_cnt[t];
+            const int ntt = t ? I.n_t1 : I.n_t0;
+            if (j >= ntt) continue;
+            if (!(ok = mbar_wait(&p_full[t], (p_par >> t) & 1u, lim, W_FWD_P))) break;
+            p_par ^= 1u << t;
             tc_fence_after();
             issue_pv(t, it_v % NS, j > 0);
-            if (j + 1 < nt[t]) {
+            if (j + 1 < ntt) {
               if (!k_ready) {
                 if (!(ok = wait_item(it_k))) break;
                 tc_fence_after();
@@ -278,7 +284,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
               }
               issue_s(t, it_k % NS);
               umma_commit(&s_full[t]);
-              if (j + 2 == nt[t]) umma_commit(&q_empty[t]);   // the last S of this Q tile
+              if (j + 2 == ntt) umma_commit(&q_empty[t]);   // the last S of this Q tile
             } else {
               umma_commit(&o_full[t]);
             }
@@ -406,29 +412,28 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       if (have_o) tc_fence_after();
       const bool has = l > 0.f;
       const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
-      const bool in_range = row < p.Lq;
-      if (in_range && p.lse != nullptr)
+      if (row < p.Lq && p.lse != nullptr)
         p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_used + log2f(l)) * LN2 : -INFINITY;
       const size_t orow = (static_cast<size_t>(b) * p.Lq + row) * p.Hq + h;
-  #pragma unroll
+#pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
         if (have_o) {
           tmem_ld_32x32b_x32(t_o + c0, ov);
         } else {
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
         }
-        if (!in_range) continue;
+        if (row >= p.Lq) continue;
         if (p.o_fp32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c0);
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(ov[4 * i]) * inv_l, __uint_as_float(ov[4 * i + 1]) * inv_l,
                                  __uint_as_float(ov[4 * i + 2]) * inv_l, __uint_as_float(ov[4 * i + 3]) * inv_l);
         } else {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D + c0);
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 wv;
             wv.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]) * inv_l, __uint_as_float(ov[8 * i + 1]) * inv_l);

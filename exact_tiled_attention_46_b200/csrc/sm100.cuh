@@ -93,6 +93,8 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
          "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// orders this thread's generic-proxy shared-memory writes before later async-proxy reads
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
