@@ -59,6 +59,30 @@ def test_fwd_matches_oracle(case):
         check_lse(l, rl)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_fwd_output_only_16_byte_aligned(D):
+    """O at a 16-byte (not 32-byte) offset: rows go out in 16-byte stores; the
+    guard elements around the output stay untouched."""
+    B, Hq, Hkv, Lq, Lk, causal = 1, 4, 2, 300, 300, True
+    x = synth.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=77)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(D)
+    ro, rl = oracle.attn_fwd(synth.as_f64(x["q"]), synth.as_f64(x["k"]), synth.as_f64(x["v"]), scale, causal)
+    n = B * Lq * Hq * D
+    for odt, off in ((torch.bfloat16, 8), (torch.float32, 4)):       # 16 bytes either way
+        buf = torch.full((n + 2 * off + 64,), 7.0, dtype=odt, device="cuda")
+        base = buf.data_ptr() % 32
+        start = off + ((32 - base) % 32) // buf.element_size()        # 32-byte aligned + 16 bytes
+        out = buf[start:start + n].view(B, Lq, Hq, D)
+        assert out.data_ptr() % 32 == 16
+        out.fill_(float("nan"))
+        _, lse = fa.fwd(q, k, v, scale=scale, causal=causal, out=out)
+        torch.cuda.synchronize()
+        check_close(f64(out), ro, bf16_output=(odt == torch.bfloat16), what=f"O {odt}")
+        check_lse(f64(lse), rl)
+        assert torch.all(buf[:start] == 7.0) and torch.all(buf[start + n:] == 7.0)
+
+
 def test_fwd_tiny_workload():
     """B1 H1 L128 D64 non-causal, scale 1/8, seed 0."""
     w = synth.WORKLOADS["tiny_fwd"]
