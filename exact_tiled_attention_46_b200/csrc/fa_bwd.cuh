@@ -15,9 +15,10 @@
 //        warp 13    tcgen05: S^T = K Q^T and dP^T = V dO^T into TMEM,
 //                   dV += P^T dO, dK += dS^T Q, dQ = dS K
 //        P^T and dS^T enter the products as bf16.  P^T = P_hi + P_lo and
-//        dS^T = dS_hi + dS_lo (each part bf16; P_hi in TMEM over S^T, the rest
-//        in swizzled shared memory); dV and dK take both parts, so that their
-//        only rounding is the fp32 accumulation, and dQ takes dS_hi.
+//        dS^T = dS_hi + dS_lo (each part bf16; P_hi and P_lo in TMEM over the
+//        S^T columns they come from, dS_hi and dS_lo in swizzled shared
+//        memory); dV and dK take both parts, so that their only rounding is the
+//        fp32 accumulation, and dQ takes dS_hi.
 //        warps 0-7  one thread per key row; warps w and w + 4 share a TMEM lane
 //                   quadrant and take 64 of the 128 query columns each (no row
 //                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
@@ -46,8 +47,7 @@ struct BwdCfg {
   static constexpr int DS_OFF = Q_OFF + NQ * 2 * TILE;
   static constexpr int DS_BYTES = 128 * 128 * 2;     // one 128 x 128 bf16 operand (128B swizzle)
   static constexpr int DSLO_OFF = DS_OFF + DS_BYTES;  // low bf16 part of dS^T
-  static constexpr int PLO_OFF = DSLO_OFF + DS_BYTES; // low bf16 part of P^T
-  static constexpr int ROW_OFF = PLO_OFF + DS_BYTES;  // stage s: lse2[128], delta[128]
+  static constexpr int ROW_OFF = DSLO_OFF + DS_BYTES; // stage s: lse2[128], delta[128]
   static constexpr int BAR_OFF = ROW_OFF + NQ * 1024;
   static constexpr int NBARS = 1 + 2 * NQ + 4 + 4 + 2;
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
@@ -230,7 +230,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, true, true);       // dQ: A = dS (MN-major), B = K (MN-major)
       const uint32_t k_base = smem_u32(smem + C::K_OFF), v_base = smem_u32(smem + C::V_OFF);
       const uint32_t q_base = smem_u32(smem + C::Q_OFF), ds_base = smem_u32(smem + C::DS_OFF);
-      const uint32_t dslo_base = smem_u32(smem + C::DSLO_OFF), plo_base = smem_u32(smem + C::PLO_OFF);
+      const uint32_t dslo_base = smem_u32(smem + C::DSLO_OFF);
+      // P^T part of queries 16kk..16kk+15 in TMEM: chunk (kk / 4, (kk % 4) / 2) of 32
+      // query columns holds P_hi in its first 16 columns and P_lo in the next 16
+      auto p_col = [](int kk) { return C::T_S + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8; };
       auto kmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
       auto mnmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + kk * 2048, 16384, 1024); };
       auto issue_s_dp = [&](int n) {
@@ -249,14 +252,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!(ok = mbar_wait(p_ready, n & 1, lim, W_BWD_P))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // dV += P_hi^T dO  (K = 128 queries; P_hi of query
-          umma_ts(tmem + C::T_DV,           // columns [64h, 64h+64) sits in TMEM columns [64h, 64h+32))
-                  tmem + C::T_S + (kk >> 2) * 64 + (kk & 3) * 8, mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
-        if (!(ok = mbar_wait(ds_ready, n & 1, lim, W_BWD_DS))) break;
-        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk)      // dV += P_hi^T dO  (K = 128 queries)
+          umma_ts(tmem + C::T_DV, tmem + p_col(kk), mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dV += P_lo^T dO
-          umma_ss(tmem + C::T_DV, kmaj(plo_base, kk), mnmaj(da, kk), ID_DVK, 1u);
+          umma_ts(tmem + C::T_DV, tmem + p_col(kk) + 16, mnmaj(da, kk), ID_DVK, 1u);
+        if (!(ok = mbar_wait(ds_ready, n & 1, lim, W_BWD_DS))) break;
+        tc_fence_after();
         const bool more = n + 1 < npairs;
         if (!C::DQ_IN_DP && more) {         // next pair's S^T, dP^T first: the compute warps start early
           if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
@@ -343,9 +345,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           fadd2(r0, r1, s0, s1, -__uint_as_float(dhi[t] << 16), -__uint_as_float(dhi[t] & 0xffff0000u));
           dlo[t] = pack_bf16x2(r0, r1);
         }
-        // P_hi of columns [c0, c0+32) -> TMEM columns hh*64 + lc*16 .. +16: inside this
-        // warp's own S columns, all of which it has already read
-        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + hh * 64 + lc * 16, phi);
+        // P_hi and P_lo of query columns [c0, c0+32) go back over the 32 S^T columns
+        // just read: P_hi to the first 16, P_lo to the next 16
+        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + c0, phi);
+        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + c0 + 16, plo);
         // the shared-memory operands of pair n - 1 must have been consumed
         if (lc == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
         // columns c0..c0+31: 4 16-byte chunks of the 128-byte row of block hh (128B swizzle)
@@ -353,7 +356,6 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int o16 = blk + (((lc * 4 + t) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(smem + C::PLO_OFF + o16) = make_uint4(plo[4 * t], plo[4 * t + 1], plo[4 * t + 2], plo[4 * t + 3]);
           *reinterpret_cast<uint4*>(smem + C::DS_OFF + o16) = make_uint4(dhi[4 * t], dhi[4 * t + 1], dhi[4 * t + 2], dhi[4 * t + 3]);
           *reinterpret_cast<uint4*>(smem + C::DSLO_OFF + o16) = make_uint4(dlo[4 * t], dlo[4 * t + 1], dlo[4 * t + 2], dlo[4 * t + 3]);
         }
