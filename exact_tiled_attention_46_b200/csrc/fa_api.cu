@@ -44,14 +44,17 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over a [B, L, H, D] bf16 tensor: dims (D, H, L, B), box (box_d, 1, box_rows, 1).
-bool map_bshd(CUtensorMap* m, const void* base, int B, int L, int H, int D, int box_d, int box_rows, bool sw128) {
+bool map_bshd(CUtensorMap* m, const void* base, int B, int L, int H, int D, int box_d, int box_rows, bool sw128,
+              bool fp32 = false) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
+  const cuuint64_t es_bytes = fp32 ? 4 : 2;
   cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(L), cuuint64_t(B)};
-  cuuint64_t strides[3] = {cuuint64_t(D) * 2, cuuint64_t(H) * D * 2, cuuint64_t(L) * H * D * 2};
+  cuuint64_t strides[3] = {cuuint64_t(D) * es_bytes, cuuint64_t(H) * D * es_bytes, cuuint64_t(L) * H * D * es_bytes};
   cuuint32_t box[4] = {cuuint32_t(box_d), 1, cuuint32_t(box_rows), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+  return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+             dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -156,12 +159,12 @@ fa_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::
 
 template <int D, bool CAUSAL>
 fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                     const fa::BwdParams& p, unsigned grid, cudaStream_t st) {
+                     const CUtensorMap& mdq, const fa::BwdParams& p, unsigned grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
   if (!launch_regs_match(fa::bwd_main_kernel<D, CAUSAL>, fa::BWD_LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(fa::bwd_main_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
-  fa::bwd_main_kernel<D, CAUSAL><<<grid, fa::BwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, mdo, p);
+  fa::bwd_main_kernel<D, CAUSAL><<<grid, fa::BwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status();
 }
 
@@ -366,9 +369,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                                                lse, lse2, delta, B, Hq, Lq, lq_pad, D);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  // the fp32 dQ accumulator takes reductions of 32-row x 32-column boxes
   if (!map_bshd(&mq, q, B, Lq, Hq, D, 64, 128, true) || !map_bshd(&mk, k, B, Lk, Hkv, D, 64, 128, true) ||
-      !map_bshd(&mv, v, B, Lk, Hkv, D, 64, 128, true) || !map_bshd(&mdo, dO, B, Lq, Hq, D, 64, 128, true))
+      !map_bshd(&mv, v, B, Lk, Hkv, D, 64, 128, true) || !map_bshd(&mdo, dO, B, Lq, Hq, D, 64, 128, true) ||
+      !map_bshd(&mdq, dq_acc, B, Lq, Hq, D, 32, 32, true, true))
     return FA_ERR_CUDA;
   fa::BwdParams p;
   p.lse2 = lse2; p.delta = delta; p.dq_acc = dq_acc; p.dk = dk; p.dv = dv;
@@ -377,8 +382,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.wait_limit_ns = g_wait_limit_ns.load();
   const unsigned grid = static_cast<unsigned>(((Lk + 127) / 128) * B * Hkv);
   fa_status s;
-  if (D == 128) s = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, p, grid, st) : launch_bwd<128, false>(mq, mk, mv, mdo, p, grid, st);
-  else s = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, p, grid, st) : launch_bwd<64, false>(mq, mk, mv, mdo, p, grid, st);
+  if (D == 128) s = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, mdq, p, grid, st) : launch_bwd<128, false>(mq, mk, mv, mdo, mdq, p, grid, st);
+  else s = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, mdq, p, grid, st) : launch_bwd<64, false>(mq, mk, mv, mdo, mdq, p, grid, st);
   if (s != FA_OK) return s;
   const size_t n = size_t(B) * Lq * Hq * D;
   const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n / 4 + 255) / 256, 148 * 16));

@@ -23,8 +23,9 @@
 //                   quadrant and take 64 of the 128 query columns each (no row
 //                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
 //        warps 8-11 one thread per query row: dQ tile from TMEM (two buffers at
-//                   D = 64) added to the fp32 accumulator with vector atomics;
-//                   at the end dK, dV out of TMEM
+//                   D = 64) into a swizzled shared-memory box per warp, added to
+//                   the fp32 accumulator by TMA reduce-add (32 rows x 32
+//                   columns per operation); at the end dK, dV out of TMEM
 //        warp 14    TMEM allocation; warp 15 idles.  The control warpgroup
 //                   (12-15) lends registers to the other three.
 //   bwd_post_kernel  dQ = scale * accumulator, converted to the output dtype.
@@ -38,7 +39,6 @@ template <int D>
 struct BwdCfg {
   static constexpr int TILE = 128 * D * 2;            // 128 rows of bf16
   static constexpr int NQ = (D == 64) ? 2 : 1;        // Q/dO stages (two do not fit at D = 128)
-  static constexpr int NDS = 1;                       // one set of P_lo / dS_hi / dS_lo buffers
   static constexpr bool DQ_IN_DP = (D == 128);        // dQ reuses the dP^T columns
   static constexpr int DQ_BUFS = DQ_IN_DP ? 1 : 2;    // dQ TMEM buffers
   static constexpr int K_OFF = 0;
@@ -48,7 +48,9 @@ struct BwdCfg {
   static constexpr int DS_BYTES = 128 * 128 * 2;     // one 128 x 128 bf16 operand (128B swizzle)
   static constexpr int DSLO_OFF = DS_OFF + DS_BYTES;  // low bf16 part of dS^T
   static constexpr int ROW_OFF = DSLO_OFF + DS_BYTES; // stage s: lse2[128], delta[128]
-  static constexpr int BAR_OFF = ROW_OFF + NQ * 1024;
+  // dQ staging: per read-out warp two 4 KB boxes (32 rows x 32 fp32, 128-byte swizzle)
+  static constexpr int DQS_OFF = ROW_OFF + NQ * 1024;
+  static constexpr int BAR_OFF = DQS_OFF + 4 * 8192;
   static constexpr int NBARS = 1 + 2 * NQ + 4 + 4 + 2;
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
   // TMEM columns
@@ -134,7 +136,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(512, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int NQ = C::NQ, KB = D / 64, NB = C::DQ_BUFS;
   extern __shared__ uint8_t smem_raw[];
@@ -376,28 +378,41 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int r = wq * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     bool ok = true;
+    uint8_t* stg = smem + C::DQS_OFF + wq * 8192;
     for (int n = 0; n < npairs; ++n) {
       const int bq = n % NB;
       if (!(ok = mbar_wait_warp(&dq_full[bq], (n / NB) & 1, lim, W_BWD_DQ))) break;
       tc_fence_after();
       const int i = i0 + n / G, hq = hkv * G + n % G;
-      const int qrow = i * 128 + r;
-      float* dst = p.dq_acc + ((size_t(b) * p.Lq + qrow) * p.Hq + hq) * D;
+      const int row0 = i * 128 + wq * 32;         // first query row of this warp's box
+      // D / 32 pieces of 32 columns, two per round (the two staging boxes)
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DQ + bq * D + c0, v);
-        if (qrow < p.Lq) {
+      for (int rd = 0; rd < D / 64; ++rd) {
+        if (lane == 0) bulk_wait_read_all();      // the boxes of the previous round are read
+        __syncwarp();
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            atomicAdd(reinterpret_cast<float4*>(dst + c0) + t,
-                      make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
-                                  __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3])));
+        for (int pc = 0; pc < 2; ++pc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DQ + bq * D + (rd * 2 + pc) * 32, v);
+          uint4* my_row = reinterpret_cast<uint4*>(stg + pc * 4096 + lane * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)            // 16-byte chunk c of row lane at c ^ (lane % 8)
+            my_row[c ^ (lane & 7)] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < p.Lq) {
+#pragma unroll
+          for (int pc = 0; pc < 2; ++pc) tma_reduce_add_4d(&tm_dq, stg + pc * 4096, (rd * 2 + pc) * 32, hq, row0, b);
+          bulk_commit_group();
         }
       }
       tc_fence_before();
       mbar_arrive(&dq_free[bq]);
     }
+    // the CTA may not exit while a reduction still reads its staging boxes
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
     const bool have = ok && npairs > 0 && mbar_wait_warp(dkv_done, 0, lim, W_BWD_DKV);
     if (have) tc_fence_after();
     const int key = j * 128 + r;

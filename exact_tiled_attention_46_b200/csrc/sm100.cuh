@@ -93,6 +93,20 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
          "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// Element-wise add of a shared-memory box into a tiled 4-D tensor (done by the
+// TMA unit at L2, bulk-group completion); rows of the box outside the tensor
+// are skipped.  The tensor map's element type (here fp32) sets the addition.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile("cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// waits until every committed bulk operation of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// waits until every committed bulk operation of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // orders this thread's generic-proxy shared-memory writes before later async-proxy reads
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
