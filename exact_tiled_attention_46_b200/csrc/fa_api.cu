@@ -376,7 +376,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
       !map_bshd(&mdq, dq_acc, B, Lq, Hq, D, 32, 32, true, true))
     return FA_ERR_CUDA;
   fa::BwdParams p;
-  p.lse2 = lse2; p.delta = delta; p.dq_acc = dq_acc; p.dk = dk; p.dv = dv;
+  p.lse2 = lse2; p.delta = delta; p.dk = dk; p.dv = dv;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.Lq_pad = lq_pad;
   p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f; p.g_fp32 = (grad_dtype == FA_FP32);
   p.wait_limit_ns = g_wait_limit_ns.load();

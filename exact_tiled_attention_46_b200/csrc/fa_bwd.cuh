@@ -62,7 +62,6 @@ struct BwdCfg {
 struct BwdParams {
   const float* lse2;     // [B*Hq, Lq_pad]  LSE * log2(e), +inf on rows without keys / padding
   const float* delta;    // [B*Hq, Lq_pad]
-  float* dq_acc;         // [B, Lq, Hq, D] fp32, zero on entry
   void* dk;              // [B, Lk, Hkv, D]
   void* dv;
   int B, Hq, Hkv, Lq, Lk, Lq_pad;
