@@ -356,7 +356,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
               const int c = half * 64 + 2 * i;
               float x0, x1, p0, p1;
               ffma2(x0, x1, s[c], s[c + 1], sl2, sl2, -msub, -msub);
-              if (use_poly && (i % 3) == 2) {
+              if (use_poly && (i % 4) == 3) {        // every fourth pair on the FMA pipe
                 exp2_poly2(x0, x1, p0, p1);
               } else {
                 p0 = ex2_approx(x0);
