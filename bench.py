@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # value (otherwise the roofline's traffic is reported as null).
 PROFILED_TRAFFIC = {
     "fwd_kernel causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
-                                  "sha256_16": "3950c0016cb9d136", "bytes": 128.374784e6 + 10.704128e6},
+                                  "sha256_16": "2afa5eb1a5e48c21", "bytes": 127.7248e6 + 10.730752e6},
 }
 
 
