@@ -64,6 +64,17 @@ constexpr float FWD_TAU = 8.0f;
 constexpr int FWD_LAUNCH_REGS = 168, FWD_SOFTMAX_REGS = 224, FWD_CTRL_REGS = 56;
 static_assert(2 * FWD_SOFTMAX_REGS + FWD_CTRL_REGS == 3 * FWD_LAUNCH_REGS, "register split must match the launch");
 constexpr float FWD_FAST_LIMIT = 65536.0f;
+// Every FWD_POLY_PERIOD-th pair of an unmasked tile can be exponentiated on the
+// FMA pipe (exp2_poly2) instead of the MUFU unit; 0 turns this off.  Measured
+// against a share of 1/3 on the causal prefill (B4 H16 L2048 D128) and long GQA
+// (B1 Hq32 Hkv8 L16384 D128) workloads: 1/2 gave -4% / -1%, 1/4 +2% / +3.5%,
+// 1/8 +3% / +5%, none +3% / +7%.  The softmax warps here are bound by their
+// issue slots rather than by the MUFU rate, so the longer polynomial sequence
+// does not pay.
+constexpr int FWD_POLY_PERIOD = 0;
+__host__ __device__ constexpr bool fwd_poly_pair(int i) {
+  return FWD_POLY_PERIOD > 0 && (i % (FWD_POLY_PERIOD > 0 ? FWD_POLY_PERIOD : 1)) == FWD_POLY_PERIOD - 1;
+}
 
 // 2^x for two lanes on the FMA pipe: x = j + f with j = round(x), f in
 // [-1/2, 1/2]; 2^f by the fitted polynomial (exp2_poly.cuh, Horner on packed
@@ -356,7 +367,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
               const int c = half * 64 + 2 * i;
               float x0, x1, p0, p1;
               ffma2(x0, x1, s[c], s[c + 1], sl2, sl2, -msub, -msub);
-              if (use_poly && (i % 4) == 3) {        // every fourth pair on the FMA pipe
+              if (use_poly && fwd_poly_pair(i)) {
                 exp2_poly2(x0, x1, p0, p1);
               } else {
                 p0 = ex2_approx(x0);
