@@ -178,10 +178,11 @@ void fa_set_wait_limit_ns(unsigned long long ns);
 fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t stream);
 
 /*
- * Self-test of the forward kernel's FMA-pipe exponential: y[i] = 2^x[i] for
- * n device floats, computed exactly as the forward computes part of its
- * probabilities (round-to-nearest split, fitted cubic, exponent add; inputs
- * below -126 give a tiny positive value).  For tests only.
+ * Self-test of the FMA-pipe exponential the forward kernel can use for part of
+ * its probabilities (off in this build: every share measured slower than the
+ * MUFU unit alone): y[i] = 2^x[i] for n device floats, computed exactly as that
+ * path does (round-to-nearest split, fitted cubic, exponent add; inputs below
+ * -126 give a tiny positive value).  For tests only.
  */
 fa_status fa_selftest_exp2_poly(const float* x, float* y, int n, fa_stream_t stream);
 
