@@ -1,5 +1,6 @@
-"""The FMA-pipe exponential of the forward kernel: fitted coefficients (CPU) and
-the device implementation against torch.exp2 (GPU)."""
+"""The FMA-pipe exponential the forward kernel can use for part of its
+probabilities (switched off in this build, FWD_POLY_PERIOD = 0): fitted
+coefficients (CPU) and the device implementation against torch.exp2 (GPU)."""
 import os
 import re
 
