@@ -110,3 +110,34 @@ def test_binding_has_no_cpu_path():
     q = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         fa.fwd(q, q, q)
+
+
+def test_static_decode_rejects_oversize_before_any_cuda_call(L):
+    # 128 sequences x 32 heads x 32 chunks of partials exceed the file-scope array
+    assert fa.decode_workspace_size(128, 32, 32768, 128) > 40 * 1024 * 1024
+    assert L.fa_decode_splitkv_static(P16, P16, P16, P16, P16, None, 128, 32, 8, 32768, 128, 0.1, 0,
+                                      None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_bwd_rejects_dtype_and_workspace_alignment(L):
+    ws = fa.bwd_workspace_size(1, 2, 128, 64)
+    base = [P16] * 9 + [1, 2, 2, 128, 128, 64, 0.125, 1, 0, 256 * 1024, ws, None]
+    a = list(base)
+    a[17] = 7                          # grad dtype
+    assert L.fa_bwd(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(base)
+    a[18] = 256 * 1024 + 16            # workspace only 16-byte aligned
+    assert L.fa_bwd(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(base)
+    a[5] = P16 + 2                     # lse not 4-byte aligned
+    assert L.fa_bwd(*a) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fwd_rejects_misaligned_lse(L):
+    assert L.fa_fwd(P16, P16, P16, P16, P16 + 2, 1, 1, 1, 8, 8, 64, 0.1, 0, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_exp2_selftest_rejects_bad_arguments(L):
+    assert L.fa_selftest_exp2_poly(None, P16, 4, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_selftest_exp2_poly(P16, P16, -1, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_selftest_exp2_poly(P16, P16, 0, None) == fa.FA_OK      # nothing to launch
