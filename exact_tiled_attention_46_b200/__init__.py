@@ -21,7 +21,7 @@ import torch
 __all__ = ["fwd", "bwd", "decode", "decode_combine", "device_status", "set_wait_limit_ns",
            "selftest_wait_timeout", "lib", "LIB_PATH", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FaError",
-           "bwd_workspace_size", "decode_workspace_size", "decode_chunk"]
+           "bwd_workspace_size", "decode_workspace_size", "decode_chunk", "launch_guard"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa46.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -44,6 +44,7 @@ _SIGNATURES = {
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
     "fa_selftest_wait_timeout": ([ctypes.c_ulonglong, _vp], _i),
     "fa_selftest_exp2_poly": ([_vp, _vp, _i, _vp], _i),
+    "fa_launch_guard": ([_i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)], _i),
 }
 
 _lib = None
@@ -210,3 +211,12 @@ def selftest_wait_timeout(wait_ns: int, device=None):
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     _check(lib().fa_selftest_wait_timeout(int(wait_ns), torch.cuda.current_stream(dev).cuda_stream),
            "fa_selftest_wait_timeout")
+
+
+def launch_guard(bwd: bool, D: int, causal: bool, query_regs: bool = True):
+    """(compiled registers or None, registers the split assumes, cached verdict) of one kernel instantiation."""
+    regs, exp, state = ctypes.c_int(-1), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().fa_launch_guard(int(bool(bwd)), int(D), int(bool(causal)),
+                                 ctypes.byref(regs) if query_regs else None, ctypes.byref(exp), ctypes.byref(state)),
+           "fa_launch_guard")
+    return (regs.value if query_regs else None), exp.value, state.value

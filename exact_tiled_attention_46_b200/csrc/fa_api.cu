@@ -120,28 +120,35 @@ __global__ void selftest_exp2_poly_kernel(const float* x, float* y, int n) {
   }
 }
 
-// The forward kernel moves registers between warpgroups (setmaxnreg); that is
-// only safe when the launch allocation per thread is exactly the one the split
-// was computed for.  A build that allocates differently is refused, never run.
+// The forward and backward kernels move registers between warpgroups
+// (setmaxnreg); that is only safe when the launch allocation per thread is
+// exactly the one the split was computed for.  A build that allocates
+// differently is refused, never run.  The verdict is kept per kernel
+// instantiation (each launch_* template instance owns its `state`), because
+// all instantiations of one kernel template share a function type.
+enum : int { REGS_UNKNOWN = 0, REGS_MATCH = 1, REGS_MISMATCH = 2 };
 template <typename F>
-bool launch_regs_match(F* func, int expected) {
-  static std::atomic<int> state{0};   // 0 unknown, 1 match, 2 mismatch
+bool launch_regs_match(F* func, int expected, std::atomic<int>& state) {
   int s = state.load();
-  if (s == 0) {
+  if (s == REGS_UNKNOWN) {
     cudaFuncAttributes a;
     if (cudaFuncGetAttributes(&a, func) != cudaSuccess) return false;
-    s = (a.numRegs == expected) ? 1 : 2;
+    s = (a.numRegs == expected) ? REGS_MATCH : REGS_MISMATCH;
     state.store(s);
   }
-  return s == 1;
+  return s == REGS_MATCH;
 }
+// Per-instantiation guard states, indexed by kernel_slot().
+std::atomic<int> g_regs_state[8];
+constexpr int kernel_slot(bool bwd, int D, bool causal) { return (bwd ? 4 : 0) + (D == 128 ? 2 : 0) + (causal ? 1 : 0); }
 
 template <int D, bool CAUSAL>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      long long grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int smem = fa::FwdCfg<D>::SMEM_BYTES;
-  if (!launch_regs_match(fa::fwd_kernel<D, CAUSAL>, fa::FWD_LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
+  if (!launch_regs_match(fa::fwd_kernel<D, CAUSAL>, fa::FWD_LAUNCH_REGS, g_regs_state[kernel_slot(false, D, CAUSAL)]))
+    return FA_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(fa::fwd_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
   fa::fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), fa::FwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, p);
   return launch_status();
@@ -162,7 +169,8 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                      const CUtensorMap& mdq, const fa::BwdParams& p, unsigned grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
-  if (!launch_regs_match(fa::bwd_main_kernel<D, CAUSAL>, fa::BWD_LAUNCH_REGS)) return FA_ERR_UNSUPPORTED;
+  if (!launch_regs_match(fa::bwd_main_kernel<D, CAUSAL>, fa::BWD_LAUNCH_REGS, g_regs_state[kernel_slot(true, D, CAUSAL)]))
+    return FA_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(fa::bwd_main_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
   fa::bwd_main_kernel<D, CAUSAL><<<grid, fa::BwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status();
@@ -406,6 +414,31 @@ fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream)
         cudaMemcpyToSymbolAsync(fa::g_fa_dev_where, &zero, 4, 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
       return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+fa_status fa_launch_guard(int bwd, int D, int causal, int* num_regs, int* expected_regs, int* state) {
+  if (D != 64 && D != 128) return FA_ERR_INVALID_ARG;
+  const int slot = kernel_slot(bwd != 0, D, causal != 0);
+  if (state) *state = g_regs_state[slot].load();
+  if (expected_regs) *expected_regs = bwd ? fa::BWD_LAUNCH_REGS : fa::FWD_LAUNCH_REGS;
+  if (num_regs) {
+    cudaFuncAttributes a;
+    cudaError_t e;
+    if (bwd) {
+      e = D == 128 ? (causal ? cudaFuncGetAttributes(&a, fa::bwd_main_kernel<128, true>)
+                             : cudaFuncGetAttributes(&a, fa::bwd_main_kernel<128, false>))
+                   : (causal ? cudaFuncGetAttributes(&a, fa::bwd_main_kernel<64, true>)
+                             : cudaFuncGetAttributes(&a, fa::bwd_main_kernel<64, false>));
+    } else {
+      e = D == 128 ? (causal ? cudaFuncGetAttributes(&a, fa::fwd_kernel<128, true>)
+                             : cudaFuncGetAttributes(&a, fa::fwd_kernel<128, false>))
+                   : (causal ? cudaFuncGetAttributes(&a, fa::fwd_kernel<64, true>)
+                             : cudaFuncGetAttributes(&a, fa::fwd_kernel<64, false>));
+    }
+    if (e != cudaSuccess) return FA_ERR_CUDA;
+    *num_regs = a.numRegs;
   }
   return FA_OK;
 }

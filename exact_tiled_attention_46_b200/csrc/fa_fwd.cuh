@@ -78,12 +78,14 @@ __host__ __device__ constexpr bool fwd_poly_pair(int i) {
 
 // 2^x for two lanes on the FMA pipe: x = j + f with j = round(x), f in
 // [-1/2, 1/2]; 2^f by the fitted polynomial (exp2_poly.cuh, Horner on packed
-// fp32); 2^j added into the exponent field.  x is clamped at -126, so the result
-// is a tiny positive number (not 0) far below 2^-126: callers use it only where
-// no entry is masked.  Relative error <= FA_EXP2_MAX_REL_ERR + fp32 rounding.
+// fp32); 2^j added into the exponent field.  x is clamped to [-126, 127]:
+// below, the result is a tiny positive number (not 0) far below 2^-126, so
+// callers use it only where no entry is masked; above, it stays the finite
+// 2^127 (never a wrapped exponent), which still trips the fast path's sum
+// limit.  Relative error <= FA_EXP2_MAX_REL_ERR + fp32 rounding in the range.
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
+  x0 = fminf(fmaxf(x0, -126.f), 127.f);
+  x1 = fminf(fmaxf(x1, -126.f), 127.f);
   constexpr float RND = 12582912.f;                  // 1.5 * 2^23: x + RND rounds x to an integer
   float t0, t1, r0, r1, f0, f1, q0, q1;
   fadd2(t0, t1, x0, x1, RND, RND);

@@ -129,7 +129,11 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
  * FA_ERR_UNSUPPORTED and launches nothing.
  *
  * The first call on a device looks up the array's address on that device
- * (with that device current); make that first call before any stream capture.
+ * (with that device current).  Under CUDA's lazy module loading that first
+ * look-up may also be what loads the library's kernels onto the device and
+ * reserves the array there, which can take time and synchronise; so make one
+ * warm-up call of this entry point on every device at start-up (before any
+ * stream capture and before the latency-critical loop).
  * All calls share the one array and it keeps the last call's contents; nothing
  * in it has to start at zero, because every partial result the combine step
  * reads is written earlier in the same call.  Calls whose kernels may overlap
@@ -176,6 +180,21 @@ void fa_set_wait_limit_ns(unsigned long long ns);
  * records FA_ERR_TIMEOUT in the device status and returns.
  */
 fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t stream);
+
+/*
+ * Register guard of the tensor-core kernels (for tests).  The forward and
+ * backward kernels hand registers between their warpgroups (setmaxnreg), which
+ * is only safe when a thread is launched with exactly the registers the split
+ * assumes; before the first launch of each kernel instantiation the library
+ * compares the compiled register count with that figure and refuses the launch
+ * (FA_ERR_UNSUPPORTED) on a mismatch.  For the instantiation (bwd, D, causal)
+ * this reports, when the pointers are not NULL: *state, that instantiation's
+ * cached verdict (0 not yet checked, 1 match, 2 mismatch; never changed by
+ * this call); *expected_regs, the figure the split assumes; *num_regs, the
+ * compiled count (queried from the runtime, which needs a GPU; pass NULL to
+ * skip).  D must be 64 or 128.  No counterpart on the pages.
+ */
+fa_status fa_launch_guard(int bwd, int D, int causal, int* num_regs, int* expected_regs, int* state);
 
 /*
  * Self-test of the FMA-pipe exponential the forward kernel can use for part of

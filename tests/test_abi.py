@@ -141,3 +141,17 @@ def test_exp2_selftest_rejects_bad_arguments(L):
     assert L.fa_selftest_exp2_poly(None, P16, 4, None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_selftest_exp2_poly(P16, P16, -1, None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_selftest_exp2_poly(P16, P16, 0, None) == fa.FA_OK      # nothing to launch
+
+
+def test_launch_guard_reports_per_instantiation_state_without_gpu(L):
+    """Before any launch every kernel instantiation's register verdict is
+    'not yet checked'; querying it (without the compiled count, which needs a
+    GPU) changes nothing."""
+    for bwd in (0, 1):
+        for D in (64, 128):
+            for causal in (0, 1):
+                regs, expected, state = fa.launch_guard(bwd, D, causal, query_regs=False)
+                assert regs is None and state == 0
+                assert expected == (128 if bwd else 168)
+    st = L.fa_launch_guard(0, 96, 0, None, None, None)
+    assert st == fa.FA_ERR_INVALID_ARG

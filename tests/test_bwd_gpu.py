@@ -9,7 +9,7 @@ import oracle
 import exact_tiled_attention_46_b200 as fa
 from exact_tiled_attention_46_b200 import inputs as synth
 
-from parity import check_close, need_gpu, f64
+from parity import check_close, check_lse, need_gpu, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -66,14 +66,28 @@ def test_bwd_empty_queries():
 
 
 def test_bwd_training_workload_sampled_heads():
-    """B8 H16 L4096 D64 causal fwd+bwd (seed 3): whole heads checked against the oracle."""
+    """B8 H16 L4096 D64 causal fwd+bwd (seed 3): on three whole heads, the
+    forward's O and LSE and the fp32 and bf16 gradients against the oracle."""
     w = synth.WORKLOADS["train_fwd_bwd"]
     x = synth.workload_inputs(w)
-    dq, dk, dv = gpu_grads(x, w.scale, w.causal, torch.float32)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.fwd(q, k, v, scale=w.scale, causal=w.causal)
+    o32, _ = fa.fwd(q, k, v, scale=w.scale, causal=w.causal, o_dtype=torch.float32)
+    grads = {}
+    for gdt in (torch.float32, torch.bfloat16):
+        grads[gdt] = [f64(t) for t in fa.bwd(q, k, v, o, do, lse, scale=w.scale, causal=w.causal, grad_dtype=gdt)]
+    torch.cuda.synchronize()
+    o, o32, lse = f64(o), f64(o32), f64(lse)
     xf = {n: synth.as_f64(x[n]) for n in x}
     for b, h in [(0, 0), (3, 9), (7, 15)]:
         sl = lambda t: t[b:b + 1, :, h:h + 1]
-        rq, rk, rv, *_ = oracle.attn_bwd(sl(xf["q"]), sl(xf["k"]), sl(xf["v"]), sl(xf["do"]), w.scale, w.causal)
-        check_close(sl(dv), rv, bf16_output=False, what=f"dV b{b} h{h}")
-        check_close(sl(dk), rk, bf16_output=False, what=f"dK b{b} h{h}")
-        check_close(sl(dq), rq, bf16_output=False, what=f"dQ b{b} h{h}")
+        rq, rk, rv, ro, rl, _ = oracle.attn_bwd(sl(xf["q"]), sl(xf["k"]), sl(xf["v"]), sl(xf["do"]), w.scale,
+                                                w.causal)
+        check_close(sl(o32), ro, bf16_output=False, what=f"O fp32 b{b} h{h}")
+        check_close(sl(o), ro, bf16_output=True, what=f"O bf16 b{b} h{h}")
+        check_lse(lse[b:b + 1, h:h + 1], rl, what=f"LSE b{b} h{h}")
+        for gdt, (dq, dk, dv) in grads.items():
+            bf = gdt == torch.bfloat16
+            check_close(sl(dv), rv, bf16_output=bf, what=f"dV {gdt} b{b} h{h}")
+            check_close(sl(dk), rk, bf16_output=bf, what=f"dK {gdt} b{b} h{h}")
+            check_close(sl(dq), rq, bf16_output=bf, what=f"dQ {gdt} b{b} h{h}")

@@ -40,15 +40,20 @@ def test_device_exp2_poly_vs_torch():
     # relative accuracy holds where 2^x is a normal float with margin (x >= -125);
     # below, the results only have to be negligibly small
     x = torch.cat([torch.linspace(-125.0, 16.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 15.75, -124.5]),
-                   torch.tensor([-126.0, -200.0, float("-inf")])])
+                   torch.tensor([-126.0, -200.0, float("-inf")]),
+                   torch.tensor([128.0, 130.5, 1000.0, float("inf")])])
     x = x.to(torch.float32).cuda()
     y = torch.empty_like(x)
     assert fa.lib().fa_selftest_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(),
                                           torch.cuda.current_stream().cuda_stream) == fa.FA_OK
     torch.cuda.synchronize()
     ref = torch.exp2(x.double())
-    ok = x >= -125.0
+    ok = (x >= -125.0) & (x <= 127.0)
     rel = ((y.double() - ref) / ref).abs()[ok]
     assert float(rel.max()) <= bound + 2.0 ** -20
-    tiny = y[~ok]
+    tiny = y[~ok & (x < 0)]
     assert torch.all(tiny >= 0) and torch.all(tiny < 2.0 ** -125)
+    # above the clamp the result stays the finite 2^127 (a large positive
+    # number that trips the fast path's sum limit), never a wrapped exponent
+    big = y[x > 127.0]
+    assert big.numel() == 4 and torch.all(torch.isfinite(big)) and torch.all(big > 2.0 ** 126)

@@ -47,6 +47,28 @@ def test_p1_rows_sum_to_one(causal, Lq, Lk):
     assert np.all(sums[..., ~allowed] == 0)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Lq,Lk", [(7, 7), (5, 9), (9, 5)])
+def test_p1_probs_match_torch_softmax(causal, Lq, Lk):
+    """attn_probs against torch's fp64 softmax of the scaled logits (an
+    independent library routine): catches a wrong scale, a wrong kv-head
+    mapping, a transposed product or a mis-aligned causal mask."""
+    rng = np.random.default_rng(11)
+    scale = 0.37
+    q, k = rnd(rng, 2, Lq, 4, 8), rnd(rng, 2, Lk, 2, 8)
+    P = oracle.attn_probs(q, k, scale, causal)
+    qt = torch.from_numpy(q).permute(0, 2, 1, 3)                     # [B, Hq, Lq, D]
+    kt = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(2, dim=1)   # head h -> kv head h // 2
+    logits = scale * qt @ kt.transpose(-1, -2)
+    i = torch.arange(Lq)[:, None]
+    j = torch.arange(Lk)[None, :]
+    allowed = (j <= i + (Lk - Lq)) if causal else torch.ones(Lq, Lk, dtype=torch.bool)
+    ref = torch.softmax(logits.masked_fill(~allowed, float("-inf")), dim=-1)
+    rows = allowed.any(-1)
+    np.testing.assert_allclose(P[:, :, rows.numpy()], ref[:, :, rows].numpy(), rtol=0, atol=1e-14)
+    assert np.all(P[:, :, ~rows.numpy()] == 0)
+
+
 # ---------------------------------------------------------------- P2 -----
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("Lq,Lk", [(6, 6), (4, 10), (10, 4), (33, 33)])
