@@ -52,13 +52,16 @@ NOMINAL_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0,
 # its units of work (see the profiles/ summaries for the captured case).
 PROFILED_TRAFFIC = {
     "fwd_kernel causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
-                                  "sha256_16": "0000000000000000", "bytes": None},
+                                  "sha256_16": "88f18afadce39b9c", "bytes": 127665408 + 9809152},
     "fwd_kernel long_gqa_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
-                                    "sha256_16": "0000000000000000", "bytes": None},
+                                    "sha256_16": "88f18afadce39b9c", "bytes": 340705024 + 98593280},
     "bwd_main_kernel train_fwd_bwd": {"sources": ("csrc/fa_bwd.cuh", "csrc/sm100.cuh"),
-                                      "sha256_16": "0000000000000000", "bytes": None},
+                                      "sha256_16": "524f18781031d1ce", "bytes": 407153920 + 225418496},
+    # captured on the first 16 sequences of the decode workload (1.359 GB of KV
+    # rows): 1.36014 GB read + 8.544 MB written, scaled by the KV bytes of a launch
     "decode_split_kernel splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
-                                           "sha256_16": "0000000000000000", "bytes_per_kv_byte": None},
+                                           "sha256_16": "130bae183ee39678",
+                                           "bytes_per_kv_byte": (1360140032 + 8544000) / 1358876672},
 }
 
 
