@@ -277,10 +277,12 @@ def section_train(fa, steps, warmup, flush, stream, peaks, peak_src, dev):
 
 
 def section_decode(fa, steps, warmup, flush, stream, peaks, peak_src, dev):
+    """Split-KV decode on the contiguous cache, then the same step with the new
+    token's K/V appended (fused KV append + decode)."""
     w = synth.WORKLOADS["splitkv_decode"]
     x = synth.decode_inputs(w.B, w.Hq, w.Hkv, w.Lk, w.D, w.seed, w.len_lo, w.len_hi, device=dev)
     q, kc, vc, sl = x["q"].to(dev), x["k_cache"], x["v_cache"], x["seqlens"].to(dev)
-    ws = torch.empty(fa.decode_workspace_size(w.B, w.Hq, w.Lk, w.D), dtype=torch.uint8, device=dev)
+    ws = torch.empty(fa.decode_workspace_size(w.B, w.Hq, w.Lk + 1, w.D), dtype=torch.uint8, device=dev)
     o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
     with nvtx("section splitkv_decode"):
@@ -289,12 +291,51 @@ def section_decode(fa, steps, warmup, flush, stream, peaks, peak_src, dev):
     t = statistics.mean(ms) * 1e-3
     kv_bytes = float(x["seqlens"].to(torch.int64).sum()) * w.Hkv * w.D * 2 * 2
     gbs = kv_bytes / t / 1e9
-    return {"workload": "splitkv_decode", "kernel": "decode_split_kernel+decode_combine_kernel", "ms": t * 1e3,
-            "ms_median": statistics.median(ms), "kv_bytes": kv_bytes, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-            "launches": 2 * steps,
-            "roofline": roofline("hbm", gbs, peaks, peak_src, "GB/s",
-                                 traffic=profiled_traffic("decode_split_kernel splitkv_decode", kv_bytes),
-                                 algorithmic_bytes=kv_bytes)}
+    res = {"workload": "splitkv_decode", "kernel": "decode_split_kernel+decode_combine_kernel", "ms": t * 1e3,
+           "ms_median": statistics.median(ms), "kv_bytes": kv_bytes, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+           "launches": 2 * steps,
+           "roofline": roofline("hbm", gbs, peaks, peak_src, "GB/s",
+                                traffic=profiled_traffic("decode_split_kernel splitkv_decode", kv_bytes),
+                                algorithmic_bytes=kv_bytes)}
+    # the same step with the new token's rows attended and written at row seqlens[b]
+    # (seqlens is not advanced, so every step does the same work)
+    kn, vn = (t_.to(dev) for t_ in synth.decode_new_rows(w.B, w.Hkv, w.D, w.seed))
+    with nvtx("section splitkv_decode_append"):
+        ms_a = time_steps(lambda: fa.decode_append(q, kn, vn, kc, vc, sl, scale=w.scale, workspace=ws, out=o,
+                                                   lse=lse), steps, warmup, flush, stream)
+    ta = statistics.mean(ms_a) * 1e-3
+    new_bytes = 2.0 * (2 * w.B * w.Hkv * w.D * 2)          # new K/V rows read once and written once
+    gbs_a = (kv_bytes + new_bytes) / ta / 1e9
+    app = {"workload": "splitkv_decode_append", "kernel": "decode_split_kernel<append>+decode_combine_kernel",
+           "ms": ta * 1e3, "ms_median": statistics.median(ms_a), "bytes": kv_bytes + new_bytes, "gbs": gbs_a,
+           "frac_hbm": gbs_a / peaks["hbm_gbs"], "launches": 2 * steps,
+           "roofline": roofline("hbm", gbs_a, peaks, peak_src, "GB/s", traffic=None,
+                                algorithmic_bytes=kv_bytes + new_bytes)}
+    return res, app
+
+
+def section_decode_paged(fa, steps, warmup, flush, stream, peaks, peak_src, dev, page_size=16):
+    """Split-KV decode from a paged cache (pool of page_size-row pages in a
+    seeded random order) holding the decode workload's rows."""
+    w = synth.WORKLOADS["splitkv_decode"]
+    x = synth.paged_decode_inputs(w.B, w.Hq, w.Hkv, w.D, page_size, w.seed, w.len_lo, w.len_hi, device=dev)
+    q, kp, vp = x["q"].to(dev), x["k_pages"], x["v_pages"]
+    tab, sl = x["page_table"].to(dev), x["seqlens"].to(dev)
+    cap = tab.shape[1] * page_size
+    ws = torch.empty(fa.decode_workspace_size(w.B, w.Hq, cap, w.D), dtype=torch.uint8, device=dev)
+    o = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    with nvtx("section splitkv_decode_paged"):
+        ms = time_steps(lambda: fa.decode_paged(q, kp, vp, tab, sl, scale=w.scale, workspace=ws, out=o, lse=lse),
+                        steps, warmup, flush, stream)
+    t = statistics.mean(ms) * 1e-3
+    kv_bytes = float(x["seqlens"].to(torch.int64).sum()) * w.Hkv * w.D * 2 * 2
+    gbs = kv_bytes / t / 1e9
+    return {"workload": f"splitkv_decode_paged{page_size}",
+            "kernel": "decode_split_kernel<paged>+decode_combine_kernel", "page_size": page_size,
+            "pool_pages": int(kp.shape[0]), "ms": t * 1e3, "ms_median": statistics.median(ms), "kv_bytes": kv_bytes,
+            "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "launches": 2 * steps,
+            "roofline": roofline("hbm", gbs, peaks, peak_src, "GB/s", traffic=None, algorithmic_bytes=kv_bytes)}
 
 
 def run_ours(args):
@@ -393,7 +434,12 @@ def run_ours(args):
         sections["long_gqa_prefill"] = section_fwd(fa, "long_gqa_prefill", sec_steps, 3, flush, stream, peaks,
                                                    peak_src, dev)
         sections["train_fwd_bwd"] = section_train(fa, sec_steps, 3, flush, stream, peaks, peak_src, dev)
-        sections["splitkv_decode"] = section_decode(fa, sec_steps, 3, flush, stream, peaks, peak_src, dev)
+        sections["splitkv_decode"], sections["splitkv_decode_append"] = section_decode(
+            fa, sec_steps, 3, flush, stream, peaks, peak_src, dev)
+        torch.cuda.empty_cache()
+        sections["splitkv_decode_paged16"] = section_decode_paged(fa, sec_steps, 3, flush, stream, peaks, peak_src,
+                                                                  dev, 16)
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

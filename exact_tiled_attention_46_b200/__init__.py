@@ -8,6 +8,8 @@ without a CUDA tensor or without the built library raises.
     o, lse = fwd(q, k, v, causal=True)            # prefill forward
     dq, dk, dv = bwd(q, k, v, o, do, lse, causal=True)
     o, lse = decode(q, k_cache, v_cache, seqlens)  # split-KV decode
+    o, lse = decode_append(q, k_new, v_new, k_cache, v_cache, seqlens)   # + KV append
+    o, lse = decode_paged(q, k_pages, v_pages, page_table, seqlens)     # paged cache
 """
 from __future__ import annotations
 
@@ -21,7 +23,8 @@ import torch
 __all__ = ["fwd", "bwd", "decode", "decode_combine", "device_status", "set_wait_limit_ns",
            "selftest_wait_timeout", "lib", "LIB_PATH", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FaError",
-           "bwd_workspace_size", "decode_workspace_size", "decode_chunk", "launch_guard"]
+           "bwd_workspace_size", "decode_workspace_size", "decode_chunk", "launch_guard", "decode_append",
+           "decode_paged"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa46.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -39,6 +42,8 @@ _SIGNATURES = {
     "fa_decode_workspace_size": ([_i, _i, _i, _i], _sz),
     "fa_decode_splitkv": ([_vp] * 6 + [_i] * 5 + [_f, _i, _vp, _sz, _vp], _i),
     "fa_decode_combine": ([_vp] * 5 + [_i] * 5 + [_vp], _i),
+    "fa_decode_append_splitkv": ([_vp] * 8 + [_i] * 5 + [_f, _i, _vp, _sz, _vp], _i),
+    "fa_decode_paged_splitkv": ([_vp] * 9 + [_i] * 7 + [_f, _i, _vp, _sz, _vp], _i),
     "fa_decode_splitkv_static": ([_vp] * 6 + [_i] * 5 + [_f, _i, _vp], _i),
     "fa_device_status": ([ctypes.POINTER(_i), ctypes.POINTER(_i), _i, _vp], _i),
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
@@ -175,6 +180,76 @@ def decode(q, k_cache, v_cache, seqlens, scale: Optional[float] = None, o_dtype=
                                    out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lmax, D, scale, _odt(out.dtype),
                                    workspace.data_ptr(), workspace.numel(), _stream(q)),
            "fa_decode_splitkv")
+    return out, lse
+
+
+def decode_append(q, k_new, v_new, k_cache, v_cache, seqlens, scale: Optional[float] = None,
+                  o_dtype=torch.bfloat16, workspace: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Decode with the new token appended: q [B,Hq,D], k_new/v_new [B,Hkv,D], caches [B,Lmax,Hkv,D].
+
+    Attends over seqlens[b] cached rows plus the new row and writes the new rows
+    into the caches at row seqlens[b]; ``seqlens`` is not advanced (add 1 after).
+    """
+    _need(q, "q", ndim=3)
+    _need(k_new, "k_new", ndim=3)
+    _need(v_new, "v_new", ndim=3)
+    _need(k_cache, "k_cache", ndim=4)
+    _need(v_cache, "v_cache", ndim=4)
+    _need(seqlens, "seqlens", dtype=torch.int32, ndim=1)
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    need = decode_workspace_size(B, Hq, Lmax + 1, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=o_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check(lib().fa_decode_append_splitkv(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(),
+                                          v_cache.data_ptr(), seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                          B, Hq, Hkv, Lmax, D, scale, _odt(out.dtype), workspace.data_ptr(),
+                                          workspace.numel(), _stream(q)),
+           "fa_decode_append_splitkv")
+    return out, lse
+
+
+def decode_paged(q, k_pages, v_pages, page_table, seqlens, k_new=None, v_new=None, scale: Optional[float] = None,
+                 o_dtype=torch.bfloat16, workspace: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Decode from a paged cache: pages [num_pages,page_size,Hkv,D], page_table int32 [B,pages_per_seq].
+
+    With k_new/v_new [B,Hkv,D] the new token is attended and appended at row
+    seqlens[b] (its page must be in the table); ``seqlens`` is not advanced.
+    """
+    _need(q, "q", ndim=3)
+    _need(k_pages, "k_pages", ndim=4)
+    _need(v_pages, "v_pages", ndim=4)
+    _need(page_table, "page_table", dtype=torch.int32, ndim=2)
+    _need(seqlens, "seqlens", dtype=torch.int32, ndim=1)
+    append = k_new is not None
+    if append:
+        _need(k_new, "k_new", ndim=3)
+        _need(v_new, "v_new", ndim=3)
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_pages.shape
+    pages_per_seq = page_table.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    need = decode_workspace_size(B, Hq, pages_per_seq * page_size + int(append), D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=o_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check(lib().fa_decode_paged_splitkv(q.data_ptr(), k_new.data_ptr() if append else None,
+                                         v_new.data_ptr() if append else None, k_pages.data_ptr(),
+                                         v_pages.data_ptr(), page_table.data_ptr(), seqlens.data_ptr(),
+                                         out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, num_pages, page_size,
+                                         pages_per_seq, D, scale, _odt(out.dtype), workspace.data_ptr(),
+                                         workspace.numel(), _stream(q)),
+           "fa_decode_paged_splitkv")
     return out, lse
 
 

@@ -154,13 +154,97 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return launch_status();
 }
 
-template <int D, int GP>
-fa_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p, dim3 grid,
+template <int D, int GP, bool PAGED, bool APPEND>
+fa_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p, unsigned grid,
                         cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   using C = fa::DecCfg<D, GP>;
-  if (!ensure_smem_attr(fa::decode_split_kernel<D, GP>, C::SMEM_BYTES, attr_done)) return FA_ERR_CUDA;
-  fa::decode_split_kernel<D, GP><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mk, mv, p);
+  if (!ensure_smem_attr(fa::decode_split_kernel<D, GP, PAGED, APPEND>, C::SMEM_BYTES, attr_done)) return FA_ERR_CUDA;
+  fa::decode_split_kernel<D, GP, PAGED, APPEND><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mk, mv, p);
+  return launch_status();
+}
+
+template <bool PAGED, bool APPEND>
+fa_status dispatch_decode(int D, int GP, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
+                          unsigned grid, cudaStream_t st) {
+  if (D == 128)
+    return GP == 4 ? launch_decode<128, 4, PAGED, APPEND>(mk, mv, p, grid, st)
+         : GP == 2 ? launch_decode<128, 2, PAGED, APPEND>(mk, mv, p, grid, st)
+                   : launch_decode<128, 1, PAGED, APPEND>(mk, mv, p, grid, st);
+  return GP == 4 ? launch_decode<64, 4, PAGED, APPEND>(mk, mv, p, grid, st)
+       : GP == 2 ? launch_decode<64, 2, PAGED, APPEND>(mk, mv, p, grid, st)
+                 : launch_decode<64, 1, PAGED, APPEND>(mk, mv, p, grid, st);
+}
+
+// One split-KV decode call, every variant: cache rows from a contiguous cache
+// (page_table == nullptr: "pages" are the sequences, page_size = Lmax) or a
+// page pool, and, when k_new != nullptr, the new token's rows attended and
+// appended.  Checks every argument before anything is launched.
+fa_status run_decode(const void* q, const void* k_new, const void* v_new, const void* k_cache, const void* v_cache,
+                     const int* page_table, const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                     int num_pages, int page_size, int pages_per_seq, int D, float scale, int o_dtype,
+                     void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  const bool paged = page_table != nullptr, append = k_new != nullptr || v_new != nullptr;
+  if (!q || !k_cache || !v_cache || !seqlens || !o || !workspace) return FA_ERR_INVALID_ARG;
+  if (append && (!k_new || !v_new)) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (num_pages <= 0 || page_size <= 0 || pages_per_seq <= 0) return FA_ERR_INVALID_ARG;
+  if (paged && page_size % 16 != 0) return FA_ERR_UNSUPPORTED;
+  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned256(workspace) ||
+      !aligned16(k_new) || !aligned16(v_new))
+    return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) != 0 || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const long long cap = static_cast<long long>(page_size) * pages_per_seq;
+  if (cap + 1 > INT_MAX) return FA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  const int GP = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+  const int HG = Hkv * (G / GP);
+  const long long keys = cap + (append ? 1 : 0);
+  const long long max_splits = (keys + kDecodeChunk - 1) / kDecodeChunk;
+  if (!fits_int(static_cast<long long>(B) * max_splits * HG) || !fits_int(static_cast<long long>(B) * Hq))
+    return FA_ERR_UNSUPPORTED;
+  if (workspace_bytes < fa_decode_workspace_size(B, Hq, static_cast<int>(keys), D)) return FA_ERR_INVALID_ARG;
+  const int sub_rows = (page_size % 32 == 0 || !paged) ? 32 : 16;
+  CUtensorMap mk, mv;
+  if (!map_bshd(&mk, k_cache, num_pages, page_size, Hkv, D, D, sub_rows, false) ||
+      !map_bshd(&mv, v_cache, num_pages, page_size, Hkv, D, D, sub_rows, false))
+    return FA_ERR_CUDA;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             align_up(size_t(B) * Hq * max_splits * D * 4, 256));
+  fa::DecParams p;
+  p.seqlens = seqlens; p.q = static_cast<const uint16_t*>(q);
+  p.k_new = static_cast<const uint16_t*>(k_new); p.v_new = static_cast<const uint16_t*>(v_new);
+  p.k_cache = static_cast<uint16_t*>(const_cast<void*>(k_cache));
+  p.v_cache = static_cast<uint16_t*>(const_cast<void*>(v_cache));
+  p.page_table = page_table;
+  p.o_part = o_part; p.lse_part = lse_part;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.max_splits = static_cast<int>(max_splits); p.chunk = kDecodeChunk;
+  p.cap = static_cast<int>(cap); p.page_size = page_size; p.pages_per_seq = pages_per_seq; p.num_pages = num_pages;
+  p.sub_rows = sub_rows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  // persistent grid: as many CTAs as fit (3 per SM), never more than there can be items
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long items = static_cast<long long>(B) * max_splits * HG;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(items, 3LL * sms));
+  fa_status s;
+  if (paged) s = append ? dispatch_decode<true, true>(D, GP, mk, mv, p, grid, st)
+                        : dispatch_decode<true, false>(D, GP, mk, mv, p, grid, st);
+  else s = append ? dispatch_decode<false, true>(D, GP, mk, mv, p, grid, st)
+                  : dispatch_decode<false, false>(D, GP, mk, mv, p, grid, st);
+  if (s != FA_OK) return s;
+  fa::CombineParams c;
+  c.o_part = o_part; c.lse_part = lse_part; c.counts = seqlens; c.o = o; c.lse = lse;
+  c.B = B; c.Hq = Hq; c.D = D; c.max_splits = static_cast<int>(max_splits); c.chunk = kDecodeChunk;
+  c.o_fp32 = (o_dtype == FA_FP32); c.cap = static_cast<int>(cap); c.append = append ? 1 : 0;
+  fa::decode_combine_kernel<<<B * Hq, 128, 0, st>>>(c);
   return launch_status();
 }
 
@@ -262,6 +346,7 @@ fa_status fa_decode_combine(const float* o_part, const float* lse_part, const in
   fa::CombineParams c;
   c.o_part = o_part; c.lse_part = lse_part; c.counts = num_splits; c.o = o; c.lse = lse;
   c.B = B; c.Hq = Hq; c.D = D; c.max_splits = max_splits; c.chunk = 0; c.o_fp32 = (o_dtype == FA_FP32);
+  c.cap = 0; c.append = 0;
   fa::decode_combine_kernel<<<B * Hq, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c);
   return launch_status();
 }
@@ -269,45 +354,29 @@ fa_status fa_decode_combine(const float* o_part, const float* lse_part, const in
 fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, void* o,
                             float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, int o_dtype,
                             void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  if (!q || !k_cache || !v_cache || !seqlens || !o || !workspace) return FA_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
-  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned256(workspace))
-    return FA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(seqlens) & 3u) != 0 || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-    return FA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  const int G = Hq / Hkv;
-  const int GP = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
-  const int max_splits = (Lmax + kDecodeChunk - 1) / kDecodeChunk;
-  if (max_splits > 65535 || Hkv * (G / GP) > 65535 || B > 65535) return FA_ERR_UNSUPPORTED;
-  if (workspace_bytes < fa_decode_workspace_size(B, Hq, Lmax, D)) return FA_ERR_INVALID_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  CUtensorMap mk, mv;
-  if (!map_bshd(&mk, k_cache, B, Lmax, Hkv, D, D, fa::DecCfg<128, 4>::T, false) ||
-      !map_bshd(&mv, v_cache, B, Lmax, Hkv, D, D, fa::DecCfg<128, 4>::T, false))
-    return FA_ERR_CUDA;
-  float* o_part = static_cast<float*>(workspace);
-  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                             align_up(size_t(B) * Hq * max_splits * D * 4, 256));
-  fa::DecParams p;
-  p.seqlens = seqlens; p.q = static_cast<const uint16_t*>(q); p.o_part = o_part; p.lse_part = lse_part;
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = Lmax; p.max_splits = max_splits; p.chunk = kDecodeChunk;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.wait_limit_ns = g_wait_limit_ns.load();
-  const dim3 grid(max_splits, Hkv * (G / GP), B);
-  fa_status s;
-  if (D == 128) s = GP == 4 ? launch_decode<128, 4>(mk, mv, p, grid, st)
-                  : GP == 2 ? launch_decode<128, 2>(mk, mv, p, grid, st) : launch_decode<128, 1>(mk, mv, p, grid, st);
-  else s = GP == 4 ? launch_decode<64, 4>(mk, mv, p, grid, st)
-         : GP == 2 ? launch_decode<64, 2>(mk, mv, p, grid, st) : launch_decode<64, 1>(mk, mv, p, grid, st);
-  if (s != FA_OK) return s;
-  fa::CombineParams c;
-  c.o_part = o_part; c.lse_part = lse_part; c.counts = seqlens; c.o = o; c.lse = lse;
-  c.B = B; c.Hq = Hq; c.D = D; c.max_splits = max_splits; c.chunk = kDecodeChunk; c.o_fp32 = (o_dtype == FA_FP32);
-  fa::decode_combine_kernel<<<B * Hq, 128, 0, st>>>(c);
-  return launch_status();
+  if (B <= 0 || Lmax <= 0) return FA_ERR_INVALID_ARG;
+  return run_decode(q, nullptr, nullptr, k_cache, v_cache, nullptr, seqlens, o, lse, B, Hq, Hkv, B, Lmax, 1, D,
+                    scale, o_dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_decode_append_splitkv(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                   void* v_cache, const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                                   int Lmax, int D, float scale, int o_dtype, void* workspace,
+                                   size_t workspace_bytes, fa_stream_t stream) {
+  if (B <= 0 || Lmax <= 0 || !k_new || !v_new) return FA_ERR_INVALID_ARG;
+  return run_decode(q, k_new, v_new, k_cache, v_cache, nullptr, seqlens, o, lse, B, Hq, Hkv, B, Lmax, 1, D, scale,
+                    o_dtype, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_decode_paged_splitkv(const void* q, const void* k_new, const void* v_new, void* k_pages,
+                                  void* v_pages, const int* page_table, const int* seqlens, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int num_pages, int page_size, int pages_per_seq, int D,
+                                  float scale, int o_dtype, void* workspace, size_t workspace_bytes,
+                                  fa_stream_t stream) {
+  if (!page_table) return FA_ERR_INVALID_ARG;
+  return run_decode(q, k_new, v_new, k_pages, v_pages, page_table, seqlens, o, lse, B, Hq, Hkv, num_pages,
+                    page_size, pages_per_seq, D, scale, o_dtype, workspace, workspace_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
@@ -406,7 +475,7 @@ fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream)
       cudaMemcpyFromSymbolAsync(&w, fa::g_fa_dev_where, 4, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (code) *code = (s == fa::FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : FA_OK;
+  if (code) *code = (s == fa::FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : (s == fa::FA_DEV_BAD_INPUT) ? FA_ERR_INVALID_ARG : FA_OK;
   if (where) *where = static_cast<int>(w);
   if (reset) {
     const uint32_t zero = 0;

@@ -1,18 +1,33 @@
-// Split-KV decode: one new query per (sequence, head) against a contiguous KV
-// cache ("Flash Attention Explained: Same Maths, Far Less Memory", section
-// "Where you actually feel it": in decode the score matrix is one row and the
-// cost is reading the cache; "Flash Attention Explained: Speed From Memory
-// Movement", "What changed in 2026": decode-phase variants).
+// Split-KV decode: one new query per (sequence, head) against a KV cache
+// ("Flash Attention Explained: Same Maths, Far Less Memory", section "Where
+// you actually feel it": in decode the score matrix is one row and the cost is
+// reading the cache; "Flash Attention Explained: Speed From Memory Movement",
+// "What changed in 2026": decode-phase variants, with its linked note on paged
+// KV caches; "FlashAttention Explained: How AI Models Process Attention Faster
+// and Use Less Memory", "FlashAttention vs. KV Cache": the cache stores the
+// past keys and values and each step adds the new token's).
 //
-// The cache of one sequence is cut into fixed chunks of keys.  A CTA owns one
-// (sequence, kv head, chunk) and the GP query heads of that kv head that it
-// packs, so each K/V byte is read from HBM once for GP heads.  Warp 4 streams
-// K and V tiles of T keys with TMA through an NS-slot mbarrier ring; warps 0-3
-// split every tile's keys, LPK = D/8 lanes per key, each lane owning 8
-// consecutive dimensions (one 16-byte chunk of a row).  Each key group keeps its own running max / running sum /
-// accumulator (log2 units); at the end of the chunk the groups and warps are
-// merged and the chunk's normalised partial output and LSE are written.  The
-// combine kernel merges the chunks of a sequence:
+// The cache of one sequence is cut into fixed chunks of keys.  A work item is
+// one (sequence, kv head, group of GP query heads, chunk); the GP heads share
+// every K/V byte read for them.  The grid is persistent: every CTA walks the
+// items blockIdx.x, blockIdx.x + gridDim.x, ... of a list that the kernel
+// derives from the device-side sequence lengths (items exist only for chunks
+// that hold keys), so the grid never carries empty CTAs and one CTA's K/V ring
+// runs on from item to item.
+//
+// Warp NW (the producer) streams K and V tiles of T keys by TMA through an
+// NS-slot mbarrier ring; the rows come from a contiguous cache [B, Lmax, Hkv,
+// D] or, in the PAGED variant, from a page pool [num_pages, page_size, Hkv, D]
+// through a per-sequence page table (one TMA box per page-aligned run of
+// sub_rows rows).  Warps 0..NW-1 split every tile's keys, LPK = D/8 lanes per
+// key, each lane owning 8 consecutive dimensions (one 16-byte chunk of a row).
+// Each key group keeps its own running max / running sum / accumulator (log2
+// units); at the end of the item the groups and warps are merged and the
+// item's normalised partial output and LSE are written.  In the APPEND variant
+// the new token's K and V rows (k_new, v_new) are attended as key seqlens[b]
+// straight from their input rows and written into the cache at row
+// seqlens[b] by one CTA, in the same launch.  The combine kernel merges the
+// chunks of a sequence:
 //   lse = ln sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s.
 #pragma once
 #include "sm100.cuh"
@@ -20,18 +35,26 @@
 namespace fa {
 
 struct DecParams {
-  const int* seqlens;      // [B] keys per sequence (device)
+  const int* seqlens;      // [B] rows already in the cache (device)
   const uint16_t* q;       // [B, Hq, D] bf16
+  const uint16_t* k_new;   // APPEND: [B, Hkv, D] bf16, the new token's rows
+  const uint16_t* v_new;
+  uint16_t* k_cache;       // APPEND: cache (contiguous) or page pool (PAGED), written at row seqlens[b]
+  uint16_t* v_cache;
+  const int* page_table;   // PAGED: [B, pages_per_seq] int32 page indices
   float* o_part;           // [B, Hq, max_splits, D]
   float* lse_part;         // [B, Hq, max_splits] (natural log)
-  int B, Hq, Hkv, Lmax, max_splits, chunk;
+  int B, Hq, Hkv, max_splits, chunk;
+  int cap;                 // rows one sequence can hold (Lmax, or pages_per_seq * page_size)
+  int page_size, pages_per_seq, num_pages;   // PAGED
+  int sub_rows;            // rows per TMA box: 32, or 16 (pages of an odd multiple of 16 rows)
   float scale_log2;
   uint64_t wait_limit_ns;
 };
 
 template <int D, int GP>
 struct DecCfg {
-  static constexpr int T = 32;                  // keys per TMA box
+  static constexpr int T = 32;                  // keys per ring slot
   static constexpr int NS = 4;                  // ring slots (K and V tile each)
   static constexpr int NW = 4;                  // consumer warps
   static constexpr int LPK = D / 8;             // lanes per key (8 dimensions each)
@@ -42,18 +65,102 @@ struct DecCfg {
   static constexpr int BAR_OFF = NS * STAGE_BYTES + MRG_FLOATS * 4;
   static constexpr int SMEM_BYTES = BAR_OFF + 2 * NS * 8 + 128;
   static constexpr int THREADS = (NW + 1) * 32;
+  static constexpr int CTAS_PER_SM = 3;
   static_assert((T / NW) % KPW == 0, "keys per warp must be a multiple of keys per step");
 };
 
 constexpr float DEC_TAU = 8.0f;
 
-enum : uint32_t { W_DEC_FULL = 0x201, W_DEC_EMPTY = 0x202, W_DEC_DRAIN = 0x203 };
+enum : uint32_t {
+  W_DEC_FULL = 0x201, W_DEC_EMPTY = 0x202, W_DEC_DRAIN = 0x203, W_DEC_PAGE = 0x204, W_DEC_APPEND_ROOM = 0x205,
+  W_DEC_APPEND_PAGE = 0x206
+};
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
   f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
   f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
   f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
   f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+// Keys attended for sequence b, and how many of them come from the cache.
+// Without APPEND: the first min(max(seqlens[b], 0), cap) cache rows.  With
+// APPEND: those rows plus the new one, when the cache has room for it (a full
+// sequence attends nothing; the combine kernel flags it).
+template <bool APPEND>
+__device__ __forceinline__ int dec_keys(const DecParams& p, int b, int& cached) {
+  const int len = max(p.seqlens[b], 0);
+  if (APPEND) {
+    if (len >= p.cap) { cached = 0; return 0; }
+    cached = len;
+    return len + 1;
+  }
+  cached = min(len, p.cap);
+  return cached;
+}
+
+// Work-list cursor.  Items are numbered sequence by sequence; sequence b owns
+// ceil(keys_b / chunk) * HG consecutive numbers (HG head groups per chunk).
+// dec_find maps item number w (non-decreasing from call to call) to its
+// sequence and its offset u inside that sequence, scanning the lengths 32
+// sequences at a time from where the previous call stopped.  All lanes of the
+// warp call it together and get the same answer; false once w is past the
+// last item.
+struct DecCursor {
+  int b;       // first sequence not yet passed
+  int base;    // items of the sequences before b
+};
+template <bool APPEND>
+__device__ __forceinline__ bool dec_find(const DecParams& p, int HG, int w, DecCursor& cur, int& b, int& u) {
+  const int lane = threadIdx.x & 31;
+  while (cur.b < p.B) {
+    const int bb = cur.b + lane;
+    int cached;
+    const int n = bb < p.B ? dec_keys<APPEND>(p, bb, cached) : 0;
+    const int c = ((n + p.chunk - 1) / p.chunk) * HG;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, bb < p.B && cur.base + incl > w);
+    if (hit) {
+      const int L = __ffs(hit) - 1;
+      cur.base += __shfl_sync(0xffffffffu, incl - c, L);
+      cur.b += L;
+      b = cur.b;
+      u = w - cur.base;
+      return true;
+    }
+    cur.base += __shfl_sync(0xffffffffu, incl, 31);
+    cur.b += 32;
+  }
+  return false;
+}
+
+// The rows of one work item.
+struct DecItem {
+  int b, hkv, hg, split;
+  int cached;     // cache rows of the sequence attended
+  int k_begin;    // first key of the chunk
+  int k_end;      // one past its last key (the new key counts)
+  int c_end;      // one past its last cache row
+  int ntiles;     // ring slots it takes
+};
+template <int T, bool APPEND>
+__device__ __forceinline__ DecItem dec_item(const DecParams& p, int HG, int GPK, int b, int u) {
+  DecItem I;
+  I.b = b;
+  I.hg = u % HG;
+  I.split = u / HG;
+  I.hkv = I.hg / GPK;
+  const int n = dec_keys<APPEND>(p, b, I.cached);
+  I.k_begin = I.split * p.chunk;
+  I.k_end = min(n, I.k_begin + p.chunk);
+  I.c_end = min(I.k_end, I.cached);
+  I.ntiles = I.c_end > I.k_begin ? (I.c_end - I.k_begin + T - 1) / T : 0;
+  return I;
 }
 
 // Sums each of the GP partial dot products over the LPK lanes of a key group
@@ -87,8 +194,8 @@ __device__ __forceinline__ void reduce_scores(float (&sc)[GP], int lane) {
   }
 }
 
-template <int D, int GP>
-__global__ void __launch_bounds__(DecCfg<D, GP>::THREADS, 3)
+template <int D, int GP, bool PAGED, bool APPEND>
+__global__ void __launch_bounds__(DecCfg<D, GP>::THREADS, DecCfg<D, GP>::CTAS_PER_SM)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const DecParams p) {
   using C = DecCfg<D, GP>;
@@ -99,16 +206,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + NS;
 
-  const int split = blockIdx.x;
-  const int groups_per_kv = (p.Hq / p.Hkv) / GP;
-  const int hkv = blockIdx.y / groups_per_kv;
-  const int hq0 = hkv * (p.Hq / p.Hkv) + (blockIdx.y % groups_per_kv) * GP;
-  const int b = blockIdx.z;
-  const int len = min(max(p.seqlens[b], 0), p.Lmax);
-  const int k_begin = split * p.chunk;
-  if (k_begin >= len) return;                   // this chunk is past the sequence: nothing to write
-  const int k_end = min(len, k_begin + p.chunk);
-  const int ntiles = (k_end - k_begin + T - 1) / T;
+  const int G = p.Hq / p.Hkv;
+  const int GPK = G / GP;                       // head groups per kv head
+  const int HG = p.Hkv * GPK;                   // head groups per chunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t lim = p.wait_limit_ns;
 
@@ -120,169 +220,283 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   if (warp == NW) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % NS;
-        if (i >= NS && !mbar_wait(&empty[s], ((i / NS) + 1) & 1, lim, W_DEC_EMPTY)) break;
-        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-        uint8_t* dst = smem + s * C::STAGE_BYTES;
-        tma_load_4d(dst, &tm_k, &full[s], 0, hkv, k_begin + i * T, b);
-        tma_load_4d(dst + C::TILE_BYTES, &tm_v, &full[s], 0, hkv, k_begin + i * T, b);
-        issued = i + 1;
+    // The whole warp walks the work list (page indices are spread over its
+    // lanes); lane 0 issues the copies.
+    if (lane == 0) { tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); }
+    DecCursor cur{0, 0};
+    int it = 0;                                 // ring slots filled so far
+    bool ok = true;
+    for (int w = blockIdx.x; ok; w += gridDim.x) {
+      int b, u;
+      if (!dec_find<APPEND>(p, HG, w, cur, b, u)) break;
+      const DecItem I = dec_item<T, APPEND>(p, HG, GPK, b, u);
+      int pg0 = 0, pg1 = 0, first_pg = 0;
+      if (PAGED && I.ntiles > 0) {
+        // a chunk spans at most 64 pages (pages hold >= 16 rows, chunks 1024)
+        first_pg = I.k_begin / p.page_size;
+        const int last_pg = (I.c_end - 1) / p.page_size;
+        const int* row = p.page_table + static_cast<size_t>(b) * p.pages_per_seq;
+        if (first_pg + lane <= last_pg) pg0 = row[first_pg + lane];
+        if (first_pg + 32 + lane <= last_pg) pg1 = row[first_pg + 32 + lane];
       }
-      for (int i = max(0, issued - NS); i < issued; ++i) mbar_wait(&full[i % NS], (i / NS) & 1, lim, W_DEC_DRAIN);
+      for (int i = 0; i < I.ntiles; ++i) {
+        const int slot = it % NS;
+        if (it >= NS && !(ok = mbar_wait_warp(&empty[slot], ((it / NS) + 1) & 1, lim, W_DEC_EMPTY))) break;
+        const int key0 = I.k_begin + i * T;
+        // boxes of sub_rows rows that hold at least one cache row of the item
+        int pages[2], rows[2];
+        uint32_t bytes = 0, use = 0;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          const int pos = key0 + s * p.sub_rows;
+          pages[s] = b;
+          rows[s] = pos;
+          if (s * p.sub_rows >= T || pos >= I.c_end) continue;
+          if (PAGED) {
+            const int idx = pos / p.page_size - first_pg;
+            pages[s] = __shfl_sync(0xffffffffu, idx < 32 ? pg0 : pg1, idx & 31);
+            rows[s] = pos % p.page_size;
+            if (pages[s] < 0 || pages[s] >= p.num_pages) {   // not in the pool: skipped and flagged
+              if (lane == 0) record_status(FA_DEV_BAD_INPUT, W_DEC_PAGE);
+              continue;
+            }
+          }
+          use |= 1u << s;
+          bytes += 2u * p.sub_rows * D * 2;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[slot], bytes);
+          uint8_t* dst = smem + slot * C::STAGE_BYTES;
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            if (!((use >> s) & 1u)) continue;
+            tma_load_4d(dst + s * p.sub_rows * D * 2, &tm_k, &full[slot], 0, I.hkv, rows[s], pages[s]);
+            tma_load_4d(dst + C::TILE_BYTES + s * p.sub_rows * D * 2, &tm_v, &full[slot], 0, I.hkv, rows[s],
+                        pages[s]);
+          }
+        }
+        ++it;
+      }
     }
+    // the CTA may not exit with copies in flight: wait for the last loads
+    if (lane == 0)
+      for (int i = max(0, it - NS); i < it; ++i) mbar_wait(&full[i % NS], (i / NS) & 1, lim, W_DEC_DRAIN);
     return;
   }
 
   // -------------------------------------------------------------- consumers --
   const int kg = lane / LPK;                    // key slot within a warp step
   const int ds = lane % LPK;                    // 16-byte chunk: dimensions 8*ds .. 8*ds+7
-  float qf[GP][8];
-#pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq0 + g) * D);
-    bf16x8_to_f32(qrow[ds], qf[g]);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;
-  }
-  float m[GP], l[GP], acc[GP][8];
-#pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    m[g] = -INFINITY; l[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-  }
-
-  // Per tile, a lane group owns KS keys (kt = warp*T/NW + st*KPW + kg).  Their
-  // scores are formed first (independent, so their reductions overlap), then
-  // one tile max per head decides a (rare) rescale, then p and the P.V update.
-  constexpr int KS = (T / NW) / KPW;
+  constexpr int KS = (T / NW) / KPW;            // keys per lane group per tile
+  DecCursor cur{0, 0};
+  int it = 0;                                   // ring slots consumed so far
   bool ok = true;
-  for (int i = 0; i < ntiles; ++i) {
-    const int s = i % NS;
-    if (!(ok = mbar_wait(&full[s], (i / NS) & 1, lim, W_DEC_FULL))) break;
-    const uint8_t* ks = smem + s * C::STAGE_BYTES;
-    const uint8_t* vs = ks + C::TILE_BYTES;
-    const int key0 = k_begin + i * T;
-    const bool full_tile = key0 + T <= k_end;
-    float sc[KS][GP];
+  for (int w = blockIdx.x;; w += gridDim.x) {
+    int b, u;
+    if (!dec_find<APPEND>(p, HG, w, cur, b, u)) break;
+    const DecItem I = dec_item<T, APPEND>(p, HG, GPK, b, u);
+    const int hq0 = I.hkv * G + (I.hg % GPK) * GP;
+
+    float qf[GP][8];
 #pragma unroll
-    for (int st = 0; st < KS; ++st) {
-      const int kt = warp * (T / NW) + st * KPW + kg;
-      float kf[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + kt * D * 2 + ds * 16), kf);
+    for (int g = 0; g < GP; ++g) {
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq0 + g) * D);
+      bf16x8_to_f32(qrow[ds], qf[g]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;
+    }
+    float m[GP], l[GP], acc[GP][8];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      m[g] = -INFINITY; l[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+    }
+
+    // Per tile, a lane group owns KS keys (kt = warp*T/NW + st*KPW + kg).  Their
+    // scores are formed first (independent, so their reductions overlap), then
+    // one tile max per head decides a (rare) rescale, then p and the P.V update.
+    for (int i = 0; ok && i < I.ntiles; ++i) {
+      const int s = it % NS;
+      if (!(ok = mbar_wait_warp(&full[s], (it / NS) & 1, lim, W_DEC_FULL))) break;
+      const uint8_t* ks = smem + s * C::STAGE_BYTES;
+      const uint8_t* vs = ks + C::TILE_BYTES;
+      const int key0 = I.k_begin + i * T;
+      const bool full_tile = key0 + T <= I.c_end;
+      float sc[KS][GP];
+#pragma unroll
+      for (int st = 0; st < KS; ++st) {
+        const int kt = warp * (T / NW) + st * KPW + kg;
+        float kf[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + kt * D * 2 + ds * 16), kf);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1], a0, a1);
+          sc[st][g] = a0 + a1;
+        }
+      }
+#pragma unroll
+      for (int st = 0; st < KS; ++st) reduce_scores<GP, LPK>(sc[st], lane);
+      if (!full_tile) {                           // rows past the item's cache rows do not count
+#pragma unroll
+        for (int st = 0; st < KS; ++st) {
+          const int kt = warp * (T / NW) + st * KPW + kg;
+          if (key0 + kt >= I.c_end) {
+#pragma unroll
+            for (int g = 0; g < GP; ++g) sc[st][g] = -INFINITY;
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float mt = sc[0][g];
+#pragma unroll
+        for (int st = 1; st < KS; ++st) mt = fmaxf(mt, sc[st][g]);
+        if (mt > m[g] + DEC_TAU) {                // false while both are -inf
+          const float a = ex2_approx(m[g] - mt);
+          l[g] *= a;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[g][e] *= a;
+          m[g] = mt;
+        }
+      }
+#pragma unroll
+      for (int st = 0; st < KS; ++st) {
+        const int kt = warp * (T / NW) + st * KPW + kg;
+        if (!full_tile && key0 + kt >= I.c_end) continue;   // never read V rows past the item's cache rows
+        float vf[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + kt * D * 2 + ds * 16), vf);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float pr = ex2_approx(sc[st][g] - m[g]);
+          l[g] += pr;
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1], acc[g][e], acc[g][e + 1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      ++it;
+    }
+
+    // the new token's key (APPEND): read from its input rows by warp 0, taken
+    // by key group 0 of that warp
+    const bool has_new = APPEND && I.cached >= I.k_begin && I.cached < I.k_end;
+    if (has_new && warp == 0 && ok) {
+      const size_t nrow = (static_cast<size_t>(b) * p.Hkv + I.hkv) * D;
+      float kf[8], vf[8], sc[GP];
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(p.k_new + nrow)[ds], kf);
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(p.v_new + nrow)[ds], vf);
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1], a0, a1);
-        sc[st][g] = a0 + a1;
+        sc[g] = a0 + a1;
       }
-    }
+      reduce_scores<GP, LPK>(sc, lane);
+      if (kg == 0) {
 #pragma unroll
-    for (int st = 0; st < KS; ++st) reduce_scores<GP, LPK>(sc[st], lane);
-    if (!full_tile) {                             // keys past the chunk end do not count
+        for (int g = 0; g < GP; ++g) {
+          if (sc[g] > m[g] + DEC_TAU) {
+            const float a = ex2_approx(m[g] - sc[g]);
+            l[g] *= a;
 #pragma unroll
-      for (int st = 0; st < KS; ++st) {
-        const int kt = warp * (T / NW) + st * KPW + kg;
-        if (key0 + kt >= k_end) {
+            for (int e = 0; e < 8; ++e) acc[g][e] *= a;
+            m[g] = sc[g];
+          }
+          const float pr = ex2_approx(sc[g] - m[g]);
+          l[g] += pr;
 #pragma unroll
-          for (int g = 0; g < GP; ++g) sc[st][g] = -INFINITY;
+          for (int e = 0; e < 8; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1], acc[g][e], acc[g][e + 1]);
         }
       }
     }
+
+    // merge the key groups of this warp (lanes ds, ds+LPK, ...)
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      float mt = sc[0][g];
-#pragma unroll
-      for (int st = 1; st < KS; ++st) mt = fmaxf(mt, sc[st][g]);
-      if (mt > m[g] + DEC_TAU) {                  // false while both are -inf
-        const float a = ex2_approx(m[g] - mt);
-        l[g] *= a;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] *= a;
-        m[g] = mt;
-      }
-    }
-#pragma unroll
-    for (int st = 0; st < KS; ++st) {
-      const int kt = warp * (T / NW) + st * KPW + kg;
-      if (!full_tile && key0 + kt >= k_end) continue;   // never read V rows past the chunk end
-      float vf[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + kt * D * 2 + ds * 16), vf);
+    for (int o = LPK; o < 32; o <<= 1) {
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        const float pr = ex2_approx(sc[st][g] - m[g]);
-        l[g] += pr;
+        const float mo = __shfl_xor_sync(0xffffffffu, m[g], o);
+        const float lo = __shfl_xor_sync(0xffffffffu, l[g], o);
+        const float mn = fmaxf(m[g], mo);
+        const float a = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - mn);
+        const float c = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mn);
+        l[g] = l[g] * a + lo * c;
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1], acc[g][e], acc[g][e + 1]);
+        for (int e = 0; e < 8; ++e) {
+          const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+          acc[g][e] = acc[g][e] * a + ao * c;
+        }
+        m[g] = mn;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-  }
+    // the previous item's readers of the merge area are done
+    asm volatile("bar.sync 1, %0;" :: "r"(NW * 32) : "memory");
+    // per-warp state to shared memory: [w][g] -> m, l, acc[D]
+    if (kg == 0) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float* dst = mrg + (warp * GP + g) * (D + 2);
+        if (ds == 0) { dst[0] = m[g]; dst[1] = l[g]; }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[2 + ds * 8 + e] = acc[g][e];
+      }
+    }
+    // every consumer warp leaves together if any of them gave up waiting
+    if (!bar_sync_and(1, NW * 32, ok)) break;
+    for (int idx = threadIdx.x; idx < GP * D; idx += NW * 32) {
+      const int g = idx / D, d = idx % D;
+      float mw[NW], mx = -INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < NW; ++w2) { mw[w2] = mrg[(w2 * GP + g) * (D + 2)]; mx = fmaxf(mx, mw[w2]); }
+      float L = 0.f, O = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < NW; ++w2) {
+        const float* src = mrg + (w2 * GP + g) * (D + 2);
+        const float a = (mw[w2] == -INFINITY) ? 0.f : ex2_approx(mw[w2] - mx);
+        L = fmaf(src[1], a, L);
+        O = fmaf(src[2 + d], a, O);
+      }
+      const size_t prow = (static_cast<size_t>(b) * p.Hq + hq0 + g) * p.max_splits + I.split;
+      p.o_part[prow * D + d] = L > 0.f ? O / L : 0.f;
+      if (d == 0) p.lse_part[prow] = L > 0.f ? (mx + log2f(L)) * LN2 : -INFINITY;
+    }
 
-  // merge the key groups of this warp (lanes ds, ds+LPK, ...)
-#pragma unroll
-  for (int o = LPK; o < 32; o <<= 1) {
-#pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[g], o);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[g], o);
-      const float mn = fmaxf(m[g], mo);
-      const float a = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - mn);
-      const float c = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mn);
-      l[g] = l[g] * a + lo * c;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], o);
-        acc[g][e] = acc[g][e] * a + ao * c;
+    // APPEND: the first head group of each kv head writes the new rows into the
+    // cache at row `cached` (nothing of this launch reads that row from the cache)
+    if (has_new && warp == 1 && (I.hg % GPK) == 0 && lane < 2 * (D / 8)) {
+      size_t rowaddr;
+      bool room = true;
+      if (PAGED) {
+        const int pg = p.page_table[static_cast<size_t>(b) * p.pages_per_seq + I.cached / p.page_size];
+        room = pg >= 0 && pg < p.num_pages;
+        rowaddr = ((static_cast<size_t>(pg) * p.page_size + I.cached % p.page_size) * p.Hkv + I.hkv) * D;
+        if (!room && lane == 0) record_status(FA_DEV_BAD_INPUT, W_DEC_APPEND_PAGE);
+      } else {
+        rowaddr = ((static_cast<size_t>(b) * p.cap + I.cached) * p.Hkv + I.hkv) * D;
       }
-      m[g] = mn;
+      if (room) {
+        const int half = lane / (D / 8), c = lane % (D / 8);
+        const size_t nrow = (static_cast<size_t>(b) * p.Hkv + I.hkv) * D;
+        const uint4 val = reinterpret_cast<const uint4*>((half ? p.v_new : p.k_new) + nrow)[c];
+        reinterpret_cast<uint4*>((half ? p.v_cache : p.k_cache) + rowaddr)[c] = val;
+      }
     }
-  }
-  // per-warp state to shared memory: [w][g] -> m, l, acc[D]
-  if (kg == 0) {
-#pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      float* dst = mrg + (warp * GP + g) * (D + 2);
-      if (ds == 0) { dst[0] = m[g]; dst[1] = l[g]; }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dst[2 + ds * 8 + e] = acc[g][e];
-    }
-  }
-  asm volatile("bar.sync 1, %0;" :: "r"(NW * 32) : "memory");
-  if (!ok) return;
-  for (int idx = threadIdx.x; idx < GP * D; idx += NW * 32) {
-    const int g = idx / D, d = idx % D;
-    float mw[NW], mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) { mw[w] = mrg[(w * GP + g) * (D + 2)]; mx = fmaxf(mx, mw[w]); }
-    float L = 0.f, O = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float* src = mrg + (w * GP + g) * (D + 2);
-      const float a = (mw[w] == -INFINITY) ? 0.f : ex2_approx(mw[w] - mx);
-      L = fmaf(src[1], a, L);
-      O = fmaf(src[2 + d], a, O);
-    }
-    const size_t prow = (static_cast<size_t>(b) * p.Hq + hq0 + g) * p.max_splits + split;
-    p.o_part[prow * D + d] = L > 0.f ? O / L : 0.f;
-    if (d == 0) p.lse_part[prow] = L > 0.f ? (mx + log2f(L)) * LN2 : -INFINITY;
   }
 }
 
 struct CombineParams {
   const float* o_part;     // [B, Hq, max_splits, D]
   const float* lse_part;   // [B, Hq, max_splits]
-  const int* counts;       // [B]: number of valid parts, or key counts when chunk > 0; may be null
+  const int* counts;       // [B]: number of valid parts, or cache lengths when chunk > 0; may be null
   void* o;                 // [B, Hq, D] bf16 or fp32
   float* lse;              // [B, Hq] or null
   int B, Hq, D, max_splits, chunk, o_fp32;
+  int cap, append;         // chunk > 0: rows a sequence can hold; 1 if a new row is attended
 };
 
 // One block per (sequence, head); thread d owns output column d.
@@ -292,7 +506,18 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const CombineParams
   int ns = p.max_splits;
   if (p.counts != nullptr) {
     const int c = max(p.counts[b], 0);
-    ns = p.chunk > 0 ? (c + p.chunk - 1) / p.chunk : c;
+    if (p.chunk > 0) {
+      int n;
+      if (p.append) {
+        n = c >= p.cap ? 0 : c + 1;
+        if (c >= p.cap && bh % p.Hq == 0 && threadIdx.x == 0) record_status(FA_DEV_BAD_INPUT, W_DEC_APPEND_ROOM);
+      } else {
+        n = min(c, p.cap);
+      }
+      ns = (n + p.chunk - 1) / p.chunk;
+    } else {
+      ns = c;
+    }
     ns = min(ns, p.max_splits);
   }
   const float* lp = p.lse_part + static_cast<size_t>(bh) * p.max_splits;

@@ -13,15 +13,19 @@ namespace fa {
 // Device-side status shared by every kernel of the library.  A kernel whose
 // bounded wait runs out stores FA_DEV_TIMEOUT (first writer wins) together
 // with a small code naming the wait, then unwinds without trapping.
-enum : uint32_t { FA_DEV_OK = 0u, FA_DEV_TIMEOUT = 1u };
+// A kernel that meets an input it cannot honour (a page index outside the
+// page pool, a sequence with no room for an appended row) stores
+// FA_DEV_BAD_INPUT the same way, skips that work and carries on.
+enum : uint32_t { FA_DEV_OK = 0u, FA_DEV_TIMEOUT = 1u, FA_DEV_BAD_INPUT = 2u };
 // (the library is one translation unit, so the words are defined here)
 __device__ uint32_t g_fa_dev_status = 0;
 __device__ uint32_t g_fa_dev_where = 0;
 
-__device__ __forceinline__ void record_timeout(uint32_t where) {
-  if (atomicCAS(&g_fa_dev_status, FA_DEV_OK, FA_DEV_TIMEOUT) == FA_DEV_OK)
+__device__ __forceinline__ void record_status(uint32_t code, uint32_t where) {
+  if (atomicCAS(&g_fa_dev_status, FA_DEV_OK, code) == FA_DEV_OK)
     atomicExch(&g_fa_dev_where, where);
 }
+__device__ __forceinline__ void record_timeout(uint32_t where) { record_status(FA_DEV_TIMEOUT, where); }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -71,6 +75,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
       return false;
     }
   }
+}
+// Named barrier over `nthreads` threads that also ANDs a predicate across them.
+__device__ __forceinline__ bool bar_sync_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+               "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+               : "=r"(r) : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads) : "memory");
+  return r != 0;
 }
 // Warp-uniform version: every lane polls, the warp agrees on the outcome, so
 // that warp-collective instructions after it are executed by all lanes or by

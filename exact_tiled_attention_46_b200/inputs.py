@@ -19,6 +19,13 @@ then round-to-nearest-even to bf16 through torch):
   that any one sequence can be regenerated alone.  Rows at or past ``len_b``
   are zero (or a caller-chosen fill).
 
+* paged decode inputs hold the same rows (same streams) in a pool of
+  fixed-size pages: the pages a sequence needs are drawn, in a seeded random
+  order, from ``default_rng([seed, 0, 2])``; unused table entries are -1 and
+  spare pool pages hold a fill value;
+* the new token's rows of a decode step with KV append come from
+  ``default_rng([seed, 0, 1])`` (K then V, [B, Hkv, D]).
+
 Tensors are laid out [B, L, H, D] (queries, keys, values, outputs) and
 [B, Lmax, Hkv, D] for the KV cache; decode queries are [B, Hq, D].
 """
@@ -133,3 +140,54 @@ def decode_inputs(B, Hq, Hkv, Lmax, D, seed, len_lo, len_hi, lens=None,
         kc[b, :n].copy_(kb)
         vc[b, :n].copy_(vb)
     return {"q": q, "k_cache": kc, "v_cache": vc, "seqlens": torch.from_numpy(lens.copy())}
+
+
+def decode_new_rows(B, Hkv, D, seed):
+    """The new token's K and V rows [B, Hkv, D] (bf16) for a decode step with append."""
+    rng = np.random.default_rng([seed, 0, 1])
+    k = rng.standard_normal((B, Hkv, D), dtype=np.float32)
+    v = rng.standard_normal((B, Hkv, D), dtype=np.float32)
+    return to_bf16(k), to_bf16(v)
+
+
+def paged_decode_inputs(B, Hq, Hkv, D, page_size, seed, len_lo, len_hi, lens=None, rows_per_seq=None,
+                        spare_pages=3, pad_value: Optional[float] = 0.0, device=None):
+    """Decode inputs in a paged cache.
+
+    Returns q [B,Hq,D], k_pages / v_pages [num_pages, page_size, Hkv, D],
+    page_table int32 [B, pages_per_seq] and seqlens int32 [B].  Sequence b's
+    rows are those of ``decode_inputs`` (same streams).  Each sequence owns
+    ceil(rows_per_seq_b / page_size) pages, where rows_per_seq_b is its length,
+    or ``rows_per_seq`` (a capacity, e.g. length + 1 to leave room for an
+    appended row); the pages are a seeded random permutation of the pool, which
+    also holds ``spare_pages`` pages no table entry names.  Table entries past a
+    sequence's pages are -1.  Pool rows that hold no cache row are
+    ``pad_value``.
+    """
+    drawn, q = decode_lengths_and_q(B, Hq, D, seed, len_lo, len_hi)
+    lens = drawn if lens is None else np.asarray(lens, dtype=np.int32)
+    need = [max(int(lens[b]), 0) if rows_per_seq is None else int(rows_per_seq[b]) for b in range(B)]
+    npg = [-(-n // page_size) for n in need]
+    pps = max(1, max(npg))
+    total = sum(npg) + spare_pages
+    order = np.random.default_rng([seed, 0, 2]).permutation(total)
+    dev = device if device is not None else "cpu"
+    kp = torch.full((total, page_size, Hkv, D), float(pad_value), dtype=torch.bfloat16, device=dev)
+    vp = torch.full((total, page_size, Hkv, D), float(pad_value), dtype=torch.bfloat16, device=dev)
+    table = np.full((B, pps), -1, dtype=np.int32)
+    nxt = 0
+    for b in range(B):
+        table[b, :npg[b]] = order[nxt:nxt + npg[b]]
+        nxt += npg[b]
+        n = int(lens[b])
+        if n <= 0:
+            continue
+        kb, vb = decode_sequence_kv(b, n, Hkv, D, seed)
+        m = -(-n // page_size)
+        idx = torch.from_numpy(table[b, :m].astype(np.int64)).to(dev)
+        for src, dst in ((kb, kp), (vb, vp)):
+            full = torch.full((m * page_size, Hkv, D), float(pad_value), dtype=torch.bfloat16)
+            full[:n] = src
+            dst.index_copy_(0, idx, full.view(m, page_size, Hkv, D).to(dev))
+    return {"q": q, "k_pages": kp, "v_pages": vp, "page_table": torch.from_numpy(table),
+            "seqlens": torch.from_numpy(lens.copy())}

@@ -112,6 +112,52 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
                             fa_stream_t stream);
 
 /*
+ * Decode with the new token's K/V appended to the cache in the same call
+ * ("FlashAttention Explained ...", section "FlashAttention vs. KV Cache": the
+ * cache keeps the past keys and values and each generated token adds its
+ * own).  k_new, v_new [B,Hkv,D] bf16 are the new token's rows.  For every
+ * sequence b with seqlens[b] < Lmax, the query attends over the seqlens[b]
+ * cached rows plus the new row (seqlens[b] + 1 keys), and the new rows are
+ * written into k_cache / v_cache at row seqlens[b] (no other cache row is
+ * touched).  seqlens is NOT advanced: the caller adds 1 after the call.  A
+ * sequence with seqlens[b] >= Lmax has no room: nothing is attended or written
+ * for it (o = 0, lse = -inf) and fa_device_status() reports
+ * FA_ERR_INVALID_ARG.  Workspace: at least fa_decode_workspace_size(B, Hq,
+ * Lmax + 1, D) bytes.  Otherwise as fa_decode_splitkv.
+ */
+fa_status fa_decode_append_splitkv(const void* q, const void* k_new, const void* v_new,
+                                   void* k_cache, void* v_cache, const int* seqlens, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                                   int o_dtype, void* workspace, size_t workspace_bytes,
+                                   fa_stream_t stream);
+
+/*
+ * Decode from a paged KV cache ("Flash Attention Explained: Speed From Memory
+ * Movement", section "What changed in 2026": decode-phase variants, and its
+ * linked note "Paged Attention: Fixing the KV Cache Memory Problem").  The
+ * rows live in a pool of fixed-size pages, k_pages / v_pages
+ * [num_pages, page_size, Hkv, D] bf16; page_table [B, pages_per_seq] int32 on
+ * the device gives, for sequence b, the pool index of its p-th page, so that
+ * cache row r of sequence b is row r % page_size of page
+ * page_table[b][r / page_size].  page_size must be a multiple of 16.  Only
+ * the table entries that cover rows below seqlens[b] (and, with append, row
+ * seqlens[b]) are read; an entry outside [0, num_pages) is never dereferenced:
+ * its rows are skipped and fa_device_status() reports FA_ERR_INVALID_ARG.
+ * k_new / v_new: NULL for plain decode over seqlens[b] rows (clamped to
+ * pages_per_seq * page_size); or the new token's rows [B,Hkv,D], attended as
+ * key seqlens[b] and written at that row, as in fa_decode_append_splitkv (the
+ * page holding that row must already be in the table).  Workspace: at least
+ * fa_decode_workspace_size(B, Hq, pages_per_seq * page_size + (append ? 1 : 0),
+ * D) bytes.  Otherwise as fa_decode_splitkv.
+ */
+fa_status fa_decode_paged_splitkv(const void* q, const void* k_new, const void* v_new,
+                                  void* k_pages, void* v_pages, const int* page_table,
+                                  const int* seqlens, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int num_pages, int page_size,
+                                  int pages_per_seq, int D, float scale, int o_dtype,
+                                  void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * Split-KV decode that allocates nothing and takes no workspace.  The pages
  * have no counterpart to this entry point; it exists for callers that cannot
  * obtain device memory at the moment they run a decode step: for example an
@@ -162,9 +208,12 @@ fa_status fa_decode_combine(const float* o_part, const float* lse_part, const in
                             int o_dtype, fa_stream_t stream);
 
 /*
- * Device status of the current device: *code receives 0 (ok) or FA_ERR_TIMEOUT
- * when some kernel's bounded wait ran out since the last reset, *where a code
- * naming the wait.  Synchronises `stream`.  reset != 0 clears the status.
+ * Device status of the current device: *code receives 0 (ok), FA_ERR_TIMEOUT
+ * when some kernel's bounded wait ran out since the last reset, or
+ * FA_ERR_INVALID_ARG when a kernel met device-side input it could not honour
+ * (a page index outside the pool, a sequence without room for an appended
+ * row) and skipped that work; *where a code naming the place (first event
+ * since the reset wins).  Synchronises `stream`.  reset != 0 clears the status.
  */
 fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream);
 

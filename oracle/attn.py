@@ -223,6 +223,68 @@ def attn_decode(q, k_cache, v_cache, seqlens, scale, pairs=None):
     return o, lse
 
 
+def paged_rows(pages, table_row, n):
+    """Rows 0..n-1 of one sequence kept in a pool of fixed-size pages.
+
+    Page "Flash Attention Explained: Speed From Memory Movement", section "What
+    changed in 2026" and its linked note on paged KV caches: a sequence's cache
+    is a list of pages from a shared pool.  ``pages`` is [num_pages, P, ...];
+    ``table_row`` lists the sequence's pages in order, so row r is row r % P of
+    page table_row[r // P].
+    """
+    P = pages.shape[1]
+    r = np.arange(int(n))
+    return pages[np.asarray(table_row)[r // P], r % P]
+
+
+def attn_decode_paged(q, k_pages, v_pages, page_table, seqlens, scale, pairs=None):
+    """Single-query attention against a paged KV cache: (O [B,Hq,D], LSE [B,Hq]).
+
+    The same definition as ``attn_decode``; only where the rows are stored
+    differs (``paged_rows``).  ``pairs`` restricts the work to a list of (b, h).
+    """
+    B, Hq, D = q.shape
+    Dv = v_pages.shape[-1]
+    o = np.zeros((B, Hq, Dv))
+    lse = np.full((B, Hq), NEG_INF)
+    for b in range(B):
+        hs = [h for (bb, h) in pairs if bb == b] if pairs is not None else list(range(Hq))
+        if not hs:
+            continue
+        n = int(seqlens[b])
+        kb = paged_rows(k_pages, page_table[b], n)[None]
+        vb = paged_rows(v_pages, page_table[b], n)[None]
+        ob, lb = attn_decode(q[b:b + 1], kb, vb, np.array([n]), scale, pairs=[(0, h) for h in hs])
+        o[b, hs], lse[b, hs] = ob[0, hs], lb[0, hs]
+    return o, lse
+
+
+def attn_decode_append(q, k_new, v_new, k_cache, v_cache, seqlens, scale):
+    """One generation step with a KV cache: (O, LSE, K cache, V cache).
+
+    Page "FlashAttention Explained: How AI Models Process Attention Faster and
+    Use Less Memory", section "FlashAttention vs. KV Cache": the cache keeps
+    the keys and values of earlier tokens and each new token adds its own.
+    Sequence b holds seqlens[b] rows; the new token's rows k_new[b], v_new[b]
+    ([B, Hkv, D]) are stored at row seqlens[b] and its query attends over all
+    seqlens[b] + 1 rows.  A sequence whose cache is full (seqlens[b] >= Lmax)
+    has no room: its cache is left as it is and it attends nothing (O = 0,
+    LSE = -inf).  Returns new cache arrays; the inputs are not modified.
+    """
+    kc = np.array(k_cache, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    Lmax = kc.shape[1]
+    lens = np.maximum(np.asarray(seqlens, dtype=np.int64), 0)
+    n = np.zeros_like(lens)
+    for b in range(kc.shape[0]):
+        if lens[b] < Lmax:
+            kc[b, lens[b]] = k_new[b]
+            vc[b, lens[b]] = v_new[b]
+            n[b] = lens[b] + 1
+    o, lse = attn_decode(q, kc, vc, n, scale)
+    return o, lse, kc, vc
+
+
 def merge_partials(o_parts, lse_parts):
     """Merge attention results over disjoint key sets.
 

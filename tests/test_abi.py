@@ -155,3 +155,46 @@ def test_launch_guard_reports_per_instantiation_state_without_gpu(L):
                 assert expected == (128 if bwd else 168)
     st = L.fa_launch_guard(0, 96, 0, None, None, None)
     assert st == fa.FA_ERR_INVALID_ARG
+
+
+def test_decode_append_rejects_bad_arguments(L):
+    # q, k_new, v_new, k_cache, v_cache, seqlens, o, lse, B, Hq, Hkv, Lmax, D, scale, o_dtype, ws, bytes, stream
+    ws = fa.decode_workspace_size(2, 4, 101, 64)
+    ok = [P16] * 7 + [None, 2, 4, 2, 100, 64, 0.1, 0, 256 * 1024, ws, None]
+    a = list(ok)
+    a[16] = fa.decode_workspace_size(2, 4, 100, 64) - 1   # too small for Lmax + 1 keys
+    assert L.fa_decode_append_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[1] = None                                            # k_new
+    assert L.fa_decode_append_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[2] = P16 + 8                                         # v_new misaligned
+    assert L.fa_decode_append_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[12] = 96
+    assert L.fa_decode_append_splitkv(*a) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_decode_paged_rejects_bad_arguments(L):
+    # q, k_new, v_new, k_pages, v_pages, table, seqlens, o, lse, B, Hq, Hkv, num_pages, page, pps, D, scale,
+    # o_dtype, ws, bytes, stream
+    ws = fa.decode_workspace_size(2, 4, 4 * 256, 64)     # capacity 1024 rows: one chunk, two with an append
+    ok = [P16, None, None, P16, P16, P16, P16, P16, None, 2, 4, 2, 10, 256, 4, 64, 0.1, 0, 256 * 1024, ws, None]
+    a = list(ok)
+    a[13] = 24                                             # page size not a multiple of 16
+    assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_UNSUPPORTED
+    a = list(ok)
+    a[5] = None                                            # no page table
+    assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[1] = P16                                             # k_new without v_new
+    assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[1], a[2] = P16, P16                                  # append needs one more key of workspace
+    assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[5] = P16 + 2                                         # misaligned table
+    assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[12] = 0                                              # empty pool
+    assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_INVALID_ARG

@@ -316,6 +316,72 @@ def test_decode_zero_length_and_padding_ignored():
     np.testing.assert_array_equal(l1, l2)
 
 
+# ------------------------------------------------ paged rows, appended KV --
+def test_paged_rows_hand_example():
+    """Pool of 4 pages of 2 rows; the sequence's pages are 3, 0, 2: its rows
+    0..4 are (page 3, row 0), (3, 1), (0, 0), (0, 1), (2, 0)."""
+    pool = np.arange(4 * 2).reshape(4, 2, 1, 1).astype(np.float64)      # value = 2 * page + row
+    rows = oracle.paged_rows(pool, [3, 0, 2], 5)
+    assert rows[:, 0, 0].tolist() == [6.0, 7.0, 0.0, 1.0, 4.0]
+
+
+@pytest.mark.parametrize("P", [1, 3, 4, 16])
+def test_paged_decode_equals_contiguous_decode(P):
+    """Any page size and any page order give the contiguous result exactly:
+    scatter a contiguous cache into a shuffled pool, read it back paged."""
+    rng = np.random.default_rng(20 + P)
+    B, Hq, Hkv, D, Lmax = 3, 4, 2, 8, 13
+    q, kc, vc = rnd(rng, B, Hq, D), rnd(rng, B, Lmax, Hkv, D), rnd(rng, B, Lmax, Hkv, D)
+    lens = np.array([13, 0, 6])
+    pps = -(-Lmax // P)
+    order = rng.permutation(B * pps + 2)                  # 2 spare pages never referenced
+    kp = np.full((B * pps + 2, P, Hkv, D), np.nan)
+    vp = np.full_like(kp, np.nan)
+    table = np.full((B, pps), -1)
+    for b in range(B):
+        for j in range(pps):
+            pg = order[b * pps + j]
+            table[b, j] = pg
+            r = np.arange(j * P, min(Lmax, (j + 1) * P))
+            kp[pg, :len(r)], vp[pg, :len(r)] = kc[b, r], vc[b, r]
+    for b in range(B):
+        np.testing.assert_array_equal(oracle.paged_rows(kp, table[b], lens[b]), kc[b, :lens[b]])
+    o1, l1 = oracle.attn_decode(q, kc, vc, lens, 0.3)
+    o2, l2 = oracle.attn_decode_paged(q, kp, vp, table, lens, 0.3)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_decode_append_equals_last_row_of_extended_causal_prefill():
+    """One step with the new token appended equals the last causal prefill row
+    of the sequence extended by that token (P8 for the appended cache), the
+    new rows land at row seqlens[b], nothing else in the cache changes, and a
+    full cache has no room."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, D, Lmax = 4, 4, 2, 8, 9
+    kc, vc = rnd(rng, B, Lmax, Hkv, D), rnd(rng, B, Lmax, Hkv, D)
+    q, kn, vn = rnd(rng, B, Hq, D), rnd(rng, B, Hkv, D), rnd(rng, B, Hkv, D)
+    lens = np.array([0, 5, 8, 9])                         # the last one is full
+    o, lse, kc2, vc2 = oracle.attn_decode_append(q, kn, vn, kc, vc, lens, 0.35)
+    for b in range(B):
+        n = lens[b]
+        if n >= Lmax:
+            assert np.all(o[b] == 0) and np.all(np.isneginf(lse[b]))
+            np.testing.assert_array_equal(kc2[b], kc[b])
+            continue
+        np.testing.assert_array_equal(kc2[b, n], kn[b])
+        np.testing.assert_array_equal(vc2[b, n], vn[b])
+        keep = np.arange(Lmax) != n
+        np.testing.assert_array_equal(kc2[b, keep], kc[b, keep])
+        kx = np.concatenate([kc[b, :n], kn[b][None]])[None]          # [1, n+1, Hkv, D]
+        vx = np.concatenate([vc[b, :n], vn[b][None]])[None]
+        qx = np.zeros((1, n + 1, Hq, D))
+        qx[0, n] = q[b]
+        of, lf = oracle.attn_fwd(qx, kx, vx, 0.35, True)
+        np.testing.assert_allclose(o[b], of[0, n], atol=1e-13)
+        np.testing.assert_allclose(lse[b], lf[0, :, n], atol=1e-13)
+
+
 # ---------------------------------------------------------------- P9 -----
 def brute_force(q, k, v, scale, causal):
     B, Lq, Hq, D = q.shape
