@@ -215,15 +215,18 @@ fa_status run_decode(const void* q, const void* k_new, const void* v_new, const 
       !map_bshd(&mv, v_cache, num_pages, page_size, Hkv, D, D, sub_rows, false))
     return FA_ERR_CUDA;
   float* o_part = static_cast<float*>(workspace);
-  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                             align_up(size_t(B) * Hq * max_splits * D * 4, 256));
+  const size_t lse_off = align_up(size_t(B) * Hq * max_splits * D * 4, 256);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off);
+  int* counter = reinterpret_cast<int*>(static_cast<char*>(workspace) + lse_off +
+                                        align_up(size_t(B) * Hq * max_splits * 4, 256));
+  if (cudaMemsetAsync(counter, 0, sizeof(int), st) != cudaSuccess) return FA_ERR_CUDA;
   fa::DecParams p;
   p.seqlens = seqlens; p.q = static_cast<const uint16_t*>(q);
   p.k_new = static_cast<const uint16_t*>(k_new); p.v_new = static_cast<const uint16_t*>(v_new);
   p.k_cache = static_cast<uint16_t*>(const_cast<void*>(k_cache));
   p.v_cache = static_cast<uint16_t*>(const_cast<void*>(v_cache));
   p.page_table = page_table;
-  p.o_part = o_part; p.lse_part = lse_part;
+  p.o_part = o_part; p.lse_part = lse_part; p.work_counter = counter;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.max_splits = static_cast<int>(max_splits); p.chunk = kDecodeChunk;
   p.cap = static_cast<int>(cap); p.page_size = page_size; p.pages_per_seq = pages_per_seq; p.num_pages = num_pages;
   p.sub_rows = sub_rows;
@@ -334,7 +337,8 @@ int fa_decode_chunk(void) { return kDecodeChunk; }
 size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int D) {
   if (B <= 0 || Hq <= 0 || Lmax < 0 || D <= 0) return 0;
   const size_t ms = std::max<size_t>(1, (size_t(Lmax) + kDecodeChunk - 1) / kDecodeChunk);
-  return align_up(size_t(B) * Hq * ms * D * 4, 256) + align_up(size_t(B) * Hq * ms * 4, 256);
+  // partial outputs, partial LSEs, the work counter of the split kernel
+  return align_up(size_t(B) * Hq * ms * D * 4, 256) + align_up(size_t(B) * Hq * ms * 4, 256) + 256;
 }
 
 fa_status fa_decode_combine(const float* o_part, const float* lse_part, const int* num_splits, void* o, float* lse,

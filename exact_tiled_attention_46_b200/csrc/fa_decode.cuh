@@ -9,11 +9,13 @@
 //
 // The cache of one sequence is cut into fixed chunks of keys.  A work item is
 // one (sequence, kv head, group of GP query heads, chunk); the GP heads share
-// every K/V byte read for them.  The grid is persistent: every CTA walks the
-// items blockIdx.x, blockIdx.x + gridDim.x, ... of a list that the kernel
-// derives from the device-side sequence lengths (items exist only for chunks
-// that hold keys), so the grid never carries empty CTAs and one CTA's K/V ring
-// runs on from item to item.
+// every K/V byte read for them.  The grid is persistent and the items are
+// handed out dynamically: the producer warp of a CTA takes the next item
+// number from a device counter (zeroed before the launch), maps it to its
+// rows through the device-side sequence lengths (items exist only for chunks
+// that hold keys) and passes it to the consumer warps through a small
+// shared-memory queue.  The grid carries no empty CTAs, CTAs that run faster
+// take more items, and one CTA's K/V ring runs on from item to item.
 //
 // Warp NW (the producer) streams K and V tiles of T keys by TMA through an
 // NS-slot mbarrier ring; the rows come from a contiguous cache [B, Lmax, Hkv,
@@ -44,6 +46,7 @@ struct DecParams {
   const int* page_table;   // PAGED: [B, pages_per_seq] int32 page indices
   float* o_part;           // [B, Hq, max_splits, D]
   float* lse_part;         // [B, Hq, max_splits] (natural log)
+  int* work_counter;       // next item number; 0 when the launch starts
   int B, Hq, Hkv, max_splits, chunk;
   int cap;                 // rows one sequence can hold (Lmax, or pages_per_seq * page_size)
   int page_size, pages_per_seq, num_pages;   // PAGED
@@ -62,8 +65,10 @@ struct DecCfg {
   static constexpr int TILE_BYTES = T * D * 2;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int MRG_FLOATS = NW * GP * (D + 2);
-  static constexpr int BAR_OFF = NS * STAGE_BYTES + MRG_FLOATS * 4;
-  static constexpr int SMEM_BYTES = BAR_OFF + 2 * NS * 8 + 128;
+  static constexpr int NI = 2;                  // item queue entries (producer -> consumers)
+  static constexpr int ITEM_OFF = NS * STAGE_BYTES + MRG_FLOATS * 4;
+  static constexpr int BAR_OFF = ITEM_OFF + 16;
+  static constexpr int SMEM_BYTES = BAR_OFF + (2 * NS + 2 * NI) * 8 + 128;
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr int CTAS_PER_SM = 3;
   static_assert((T / NW) % KPW == 0, "keys per warp must be a multiple of keys per step");
@@ -73,7 +78,7 @@ constexpr float DEC_TAU = 8.0f;
 
 enum : uint32_t {
   W_DEC_FULL = 0x201, W_DEC_EMPTY = 0x202, W_DEC_DRAIN = 0x203, W_DEC_PAGE = 0x204, W_DEC_APPEND_ROOM = 0x205,
-  W_DEC_APPEND_PAGE = 0x206
+  W_DEC_APPEND_PAGE = 0x206, W_DEC_ITEM = 0x207, W_DEC_ITEM_EMPTY = 0x208
 };
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
@@ -101,9 +106,10 @@ __device__ __forceinline__ int dec_keys(const DecParams& p, int b, int& cached) 
 
 // Work-list cursor.  Items are numbered sequence by sequence; sequence b owns
 // ceil(keys_b / chunk) * HG consecutive numbers (HG head groups per chunk).
-// dec_find maps item number w (non-decreasing from call to call) to its
-// sequence and its offset u inside that sequence, scanning the lengths 32
-// sequences at a time from where the previous call stopped.  All lanes of the
+// dec_find maps item number w (non-decreasing from call to call: a CTA's
+// numbers come from a counter that only grows) to its sequence and its offset
+// u inside that sequence, scanning the lengths 32 sequences at a time from
+// where the previous call stopped.  All lanes of the
 // warp call it together and get the same answer; false once w is past the
 // last item.
 struct DecCursor {
@@ -203,8 +209,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   float* mrg = reinterpret_cast<float*>(smem + NS * C::STAGE_BYTES);
+  volatile int* item_w = reinterpret_cast<volatile int*>(smem + C::ITEM_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + NS;
+  uint64_t* item_full = empty + NS;             // [NI] an item number was posted
+  uint64_t* item_empty = item_full + C::NI;     // [NI] every consumer warp has read it
 
   const int G = p.Hq / p.Hkv;
   const int GPK = G / GP;                       // head groups per kv head
@@ -214,6 +223,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], NW); }
+    for (int i = 0; i < C::NI; ++i) { mbar_init(&item_full[i], 1); mbar_init(&item_empty[i], NW); }
     fence_mbar_init();
   }
   __syncthreads();
@@ -225,10 +235,24 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     if (lane == 0) { tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v); }
     DecCursor cur{0, 0};
     int it = 0;                                 // ring slots filled so far
+    int ni = 0;                                 // items posted to the consumers
     bool ok = true;
-    for (int w = blockIdx.x; ok; w += gridDim.x) {
-      int b, u;
-      if (!dec_find<APPEND>(p, HG, w, cur, b, u)) break;
+    while (ok) {
+      int w = 0;
+      if (lane == 0) w = atomicAdd(p.work_counter, 1);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      int b = 0, u = 0;
+      const bool more = dec_find<APPEND>(p, HG, w, cur, b, u);
+      // post the item number (-1: no more items) to the consumers
+      const int qs = ni % C::NI;
+      if (ni >= C::NI && !(ok = mbar_wait_warp(&item_empty[qs], ((ni / C::NI) + 1) & 1, lim, W_DEC_ITEM_EMPTY)))
+        break;
+      if (lane == 0) {
+        item_w[qs] = more ? w : -1;
+        mbar_arrive(&item_full[qs]);            // release: the consumers' wait sees the number
+      }
+      ++ni;
+      if (!more) break;
       const DecItem I = dec_item<T, APPEND>(p, HG, GPK, b, u);
       int pg0 = 0, pg1 = 0, first_pg = 0;
       if (PAGED && I.ntiles > 0) {
@@ -290,10 +314,20 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   constexpr int KS = (T / NW) / KPW;            // keys per lane group per tile
   DecCursor cur{0, 0};
   int it = 0;                                   // ring slots consumed so far
+  int ni = 0;                                   // items taken from the queue
   bool ok = true;
-  for (int w = blockIdx.x;; w += gridDim.x) {
+  for (;;) {
+    const int qs = ni % C::NI;
+    ok = mbar_wait_warp(&item_full[qs], (ni / C::NI) & 1, lim, W_DEC_ITEM);
+    const int w = ok ? item_w[qs] : -1;
+    __syncwarp();
+    if (ok && lane == 0) mbar_arrive(&item_empty[qs]);
+    ++ni;
+    // every consumer warp leaves together, at the end of the list or if any of
+    // them gave up waiting (the barriers below need all of them)
+    if (!bar_sync_and(1, NW * 32, ok && w >= 0)) break;
     int b, u;
-    if (!dec_find<APPEND>(p, HG, w, cur, b, u)) break;
+    dec_find<APPEND>(p, HG, w, cur, b, u);
     const DecItem I = dec_item<T, APPEND>(p, HG, GPK, b, u);
     const int hq0 = I.hkv * G + (I.hg % GPK) * GP;
 
