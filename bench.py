@@ -241,6 +241,30 @@ def section_fwd(fa, name, steps, warmup, flush, stream, peaks, peak_src, dev):
                                  traffic=profiled_traffic(f"fwd_kernel {name}"), algorithmic_bytes=fwd_bytes(w))}
 
 
+def section_fwd_fp8(fa, name, steps, warmup, flush, stream, peaks, peak_src, dev):
+    """The forward on the same draws quantized to e4m3 (per-tensor scales);
+    its peak is the measured bf16 one times the nominal fp8:bf16 ratio (2)."""
+    w = synth.WORKLOADS[name]
+    x = synth.prefill_inputs_fp8(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.D, w.seed, q_boost_heads=w.q_boost_heads)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty((w.B, w.Lq, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+    with nvtx(f"section {name}_fp8"):
+        ms = time_steps(lambda: fa.fwd_fp8(q, k, v, x["q_scale"], x["k_scale"], x["v_scale"], scale=w.scale,
+                                           causal=w.causal, out=o, lse=lse), steps, warmup, flush, stream)
+    t = statistics.mean(ms) * 1e-3
+    tf = fwd_flops(w) / t / 1e12
+    fp8_peaks = dict(peaks)
+    fp8_peaks["bf16_tflops"] = 2.0 * peaks["bf16_tflops"]
+    r = roofline("tensor", tf, fp8_peaks, peak_src, "TFLOP/s", traffic=None,
+                 algorithmic_bytes=fwd_bytes(w) - (w.B * w.Lq * w.Hq * w.D + 2 * w.B * w.Lk * w.Hkv * w.D))
+    r["peak_source"] = f"{peak_src} bf16 burst x 2 (nominal fp8:bf16 ratio)"
+    r["peak_nominal"] = 2.0 * NOMINAL_PEAKS["bf16_tflops"]
+    r["frac_nominal"] = tf / r["peak_nominal"]
+    return {"workload": f"{name}_fp8", "kernel": "fwd_kernel<fp8>", "dtype": "e4m3 in, fp32 accumulate",
+            "ms": t * 1e3, "ms_median": statistics.median(ms), "tflops": tf, "launches": steps, "roofline": r}
+
+
 def section_train(fa, steps, warmup, flush, stream, peaks, peak_src, dev):
     w = synth.WORKLOADS["train_fwd_bwd"]
     x = synth.workload_inputs(w)
@@ -433,6 +457,8 @@ def run_ours(args):
         sec_steps = max(3, min(args.steps, 20))
         sections["long_gqa_prefill"] = section_fwd(fa, "long_gqa_prefill", sec_steps, 3, flush, stream, peaks,
                                                    peak_src, dev)
+        sections["causal_prefill_fp8"] = section_fwd_fp8(fa, "causal_prefill", sec_steps, 3, flush, stream, peaks,
+                                                         peak_src, dev)
         sections["train_fwd_bwd"] = section_train(fa, sec_steps, 3, flush, stream, peaks, peak_src, dev)
         sections["splitkv_decode"], sections["splitkv_decode_append"] = section_decode(
             fa, sec_steps, 3, flush, stream, peaks, peak_src, dev)

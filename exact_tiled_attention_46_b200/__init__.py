@@ -24,7 +24,7 @@ __all__ = ["fwd", "bwd", "decode", "decode_combine", "device_status", "set_wait_
            "selftest_wait_timeout", "lib", "LIB_PATH", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FaError",
            "bwd_workspace_size", "decode_workspace_size", "decode_chunk", "launch_guard", "decode_append",
-           "decode_paged"]
+           "decode_paged", "fwd_fp8"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa46.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -36,6 +36,7 @@ _SIGNATURES = {
     "fa_status_string": ([_i], ctypes.c_char_p),
     "fa_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp], _i),
+    "fa_fwd_fp8": ([_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp], _i),
     "fa_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp] * 9 + [_i] * 6 + [_f, _i, _i, _vp, _sz, _vp], _i),
     "fa_decode_chunk": ([], _i),
@@ -121,6 +122,28 @@ def fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, o_dtype=to
     _check(lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                            B, Hq, Hkv, Lq, Lk, D, scale, int(bool(causal)), _odt(out.dtype), _stream(q)),
            "fa_fwd")
+    return out, lse
+
+
+def fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, scale: Optional[float] = None,
+            causal: bool = False, o_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None):
+    """Forward attention on e4m3 inputs (torch.float8_e4m3fn, values = e4m3 * their scale) -> (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dtype=torch.float8_e4m3fn, ndim=4)
+    B, Lq, Hq, D = q.shape
+    _, Lk, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Lq, Hq, D), dtype=o_dtype, device=q.device)
+    _need(out, "out", dtype=None, ndim=4)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    _need(lse, "lse", dtype=torch.float32, ndim=3)
+    _check(lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale), float(v_scale),
+                            out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lq, Lk, D, scale, int(bool(causal)),
+                            _odt(out.dtype), _stream(q)),
+           "fa_fwd_fp8")
     return out, lse
 
 

@@ -43,17 +43,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4-D map over a [B, L, H, D] bf16 tensor: dims (D, H, L, B), box (box_d, 1, box_rows, 1).
+// 4-D map over a [B, L, H, D] tensor (bf16; fp32 or single bytes when asked):
+// dims (D, H, L, B), box (box_d, 1, box_rows, 1).
 bool map_bshd(CUtensorMap* m, const void* base, int B, int L, int H, int D, int box_d, int box_rows, bool sw128,
-              bool fp32 = false) {
+              bool fp32 = false, bool bytes = false) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
-  const cuuint64_t es_bytes = fp32 ? 4 : 2;
+  const cuuint64_t es_bytes = fp32 ? 4 : bytes ? 1 : 2;
   cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(L), cuuint64_t(B)};
   cuuint64_t strides[3] = {cuuint64_t(D) * es_bytes, cuuint64_t(H) * D * es_bytes, cuuint64_t(L) * H * D * es_bytes};
   cuuint32_t box[4] = {cuuint32_t(box_d), 1, cuuint32_t(box_rows), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+  const CUtensorMapDataType dt = fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(m, dt, 4, const_cast<void*>(base),
              dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -139,18 +142,21 @@ bool launch_regs_match(F* func, int expected, std::atomic<int>& state) {
   return s == REGS_MATCH;
 }
 // Per-instantiation guard states, indexed by kernel_slot().
-std::atomic<int> g_regs_state[8];
-constexpr int kernel_slot(bool bwd, int D, bool causal) { return (bwd ? 4 : 0) + (D == 128 ? 2 : 0) + (causal ? 1 : 0); }
+std::atomic<int> g_regs_state[10];
+constexpr int kernel_slot(bool bwd, int D, bool causal, bool fp8 = false) {
+  return fp8 ? 8 + (causal ? 1 : 0) : (bwd ? 4 : 0) + (D == 128 ? 2 : 0) + (causal ? 1 : 0);
+}
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      long long grid, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
-  constexpr int smem = fa::FwdCfg<D>::SMEM_BYTES;
-  if (!launch_regs_match(fa::fwd_kernel<D, CAUSAL>, fa::FWD_LAUNCH_REGS, g_regs_state[kernel_slot(false, D, CAUSAL)]))
+  constexpr int smem = fa::FwdCfg<D, FP8>::SMEM_BYTES;
+  if (!launch_regs_match(fa::fwd_kernel<D, CAUSAL, FP8>, fa::FWD_LAUNCH_REGS,
+                         g_regs_state[kernel_slot(false, D, CAUSAL, FP8)]))
     return FA_ERR_UNSUPPORTED;
-  if (!ensure_smem_attr(fa::fwd_kernel<D, CAUSAL>, smem, attr_done)) return FA_ERR_CUDA;
-  fa::fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), fa::FwdCfg<D>::THREADS, smem, st>>>(mq, mk, mv, p);
+  if (!ensure_smem_attr(fa::fwd_kernel<D, CAUSAL, FP8>, smem, attr_done)) return FA_ERR_CUDA;
+  fa::fwd_kernel<D, CAUSAL, FP8><<<static_cast<unsigned>(grid), fa::FwdCfg<D, FP8>::THREADS, smem, st>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -318,6 +324,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
   p.o = o; p.lse = lse; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk;
   p.num_pairs = static_cast<int>(pairs);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_scale = 1.f;
   p.o_fp32 = (o_dtype == FA_FP32);
   p.wait_limit_ns = g_wait_limit_ns.load();
   const int sms = sm_count();
@@ -325,6 +332,46 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
   const long long grid = items < sms ? items : sms;
   if (D == 128) return causal ? launch_fwd<128, true>(mq, mk, mv, p, grid, st) : launch_fwd<128, false>(mq, mk, mv, p, grid, st);
   return causal ? launch_fwd<64, true>(mq, mk, mv, p, grid, st) : launch_fwd<64, false>(mq, mk, mv, p, grid, st);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale, float v_scale,
+                     void* o, float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int causal,
+                     int o_dtype, fa_stream_t stream) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq < 0 || Lk < 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (Lq > 0 && (!q || !o)) return FA_ERR_INVALID_ARG;
+  if (Lq > 0 && Lk > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
+  if (!scale_ok(scale) || !scale_ok(q_scale) || !scale_ok(k_scale) || !scale_ok(v_scale)) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (D != 128) return FA_ERR_UNSUPPORTED;
+  const long long pairs = (static_cast<long long>(Lq) + 255) / 256;
+  const long long items = pairs * B * Hq;
+  if (!fits_int(items) || !fits_int(static_cast<long long>(B) * Hq)) return FA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Lq == 0) return FA_OK;
+  if (Lk == 0) {
+    const size_t n_o = size_t(B) * Lq * Hq * D, n_l = size_t(B) * Hq * Lq;
+    fill_empty_rows_kernel<<<296, 256, 0, st>>>(o, lse, n_o, n_l, o_dtype == FA_FP32);
+    return launch_status();
+  }
+  CUtensorMap mq, mk, mv;
+  if (!map_bshd(&mq, q, B, Lq, Hq, D, 128, 128, true, false, true) ||
+      !map_bshd(&mk, k, B, Lk, Hkv, D, 128, 128, true, false, true) ||
+      !map_bshd(&mv, v, B, Lk, Hkv, D, 128, 128, true, false, true))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = o; p.lse = lse; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk;
+  p.num_pairs = static_cast<int>(pairs);
+  p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  p.o_scale = v_scale;
+  p.o_fp32 = (o_dtype == FA_FP32);
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long grid = items < sms ? items : sms;
+  return causal ? launch_fwd<128, true, true>(mq, mk, mv, p, grid, st)
+                : launch_fwd<128, false, true>(mq, mk, mv, p, grid, st);
 }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
@@ -492,14 +539,19 @@ fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream)
 }
 
 fa_status fa_launch_guard(int bwd, int D, int causal, int* num_regs, int* expected_regs, int* state) {
-  if (D != 64 && D != 128) return FA_ERR_INVALID_ARG;
-  const int slot = kernel_slot(bwd != 0, D, causal != 0);
+  // D = -128 names the e4m3 forward
+  const bool fp8 = (D == -128 && !bwd);
+  if (D != 64 && D != 128 && !fp8) return FA_ERR_INVALID_ARG;
+  const int slot = kernel_slot(bwd != 0, D, causal != 0, fp8);
   if (state) *state = g_regs_state[slot].load();
   if (expected_regs) *expected_regs = bwd ? fa::BWD_LAUNCH_REGS : fa::FWD_LAUNCH_REGS;
   if (num_regs) {
     cudaFuncAttributes a;
     cudaError_t e;
-    if (bwd) {
+    if (fp8) {
+      e = causal ? cudaFuncGetAttributes(&a, fa::fwd_kernel<128, true, true>)
+                 : cudaFuncGetAttributes(&a, fa::fwd_kernel<128, false, true>);
+    } else if (bwd) {
       e = D == 128 ? (causal ? cudaFuncGetAttributes(&a, fa::bwd_main_kernel<128, true>)
                              : cudaFuncGetAttributes(&a, fa::bwd_main_kernel<128, false>))
                    : (causal ? cudaFuncGetAttributes(&a, fa::bwd_main_kernel<64, true>)

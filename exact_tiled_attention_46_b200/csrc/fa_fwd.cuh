@@ -36,15 +36,20 @@ struct FwdParams {
   float* lse;              // [B, Hq, Lq] or nullptr
   int B, Hq, Hkv, Lq, Lk;
   int num_pairs;           // ceil(Lq / 256)
-  float scale_log2;        // scale * log2(e)
+  float scale_log2;        // scale * log2(e) (e4m3 inputs: times the Q and K scales)
+  float o_scale;           // multiplies O (e4m3 inputs: the V scale; else 1)
   int o_fp32;
   uint64_t wait_limit_ns;
 };
 
-template <int D>
+// FP8: Q, K, V are e4m3 (one byte per element) and both products run as
+// kind::f8f6f4 (D = 128 only: one 128-byte swizzle column per row).
+template <int D, bool FP8 = false>
 struct FwdCfg {
-  static constexpr int TILE_BYTES = 128 * D * 2;       // one 128-row bf16 tile
-  static constexpr int NS = (D == 128) ? 4 : 8;        // K/V slots
+  static constexpr int ES = FP8 ? 1 : 2;               // bytes per input element
+  static constexpr int TILE_BYTES = 128 * D * ES;      // one 128-row tile
+  static constexpr int KB = D * ES / 128;              // 128-byte column blocks per row (one TMA box each)
+  static constexpr int NS = (TILE_BYTES == 32768) ? 4 : 8;   // K/V slots
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
@@ -99,6 +104,13 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
   p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
+// The e4m3 path stores P scaled by 2^FWD_F8_P_LOG2 against the reference max
+// and moves the reference whenever a tile max exceeds it by more than
+// FWD_F8_TAU, so every stored value is at most 2^(8 + 0.75) = 431 (e4m3's
+// largest finite value is 448) and values down to 2^-17 of the row's largest
+// stay representable.
+constexpr float FWD_F8_P_LOG2 = 8.0f, FWD_F8_TAU = 0.75f;
+
 enum : uint32_t {
   W_FWD_Q = 0x101, W_FWD_KV_EMPTY = 0x102, W_FWD_KV_FULL = 0x103, W_FWD_P = 0x104,
   W_FWD_S = 0x105, W_FWD_O = 0x106, W_FWD_DONE = 0x107, W_FWD_DRAIN = 0x108, W_FWD_Q_EMPTY = 0x109
@@ -147,13 +159,15 @@ __device__ __forceinline__ int fwd_item_index(int r) {
   return r * G + ((r & 1) ? (G - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x));
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = FwdCfg<D>;
+  static_assert(!FP8 || D == 128, "the e4m3 path is built for D = 128");
+  using C = FwdCfg<D, FP8>;
   constexpr int NS = C::NS;
-  constexpr int KB = D / 64;                       // 64-column (128-byte) blocks per row
+  constexpr int KB = C::KB;                        // 128-byte column blocks per row
+  constexpr int BOX_COLS = 128 / C::ES;            // elements per 128-byte block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -209,7 +223,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           if (((q_loaded >> t) & 1u) && !(ok = mbar_wait(&q_empty[t], ((q_par >> t) & 1u) ^ 1u, lim, W_FWD_Q_EMPTY))) break;
           mbar_arrive_expect_tx(&q_full[t], C::TILE_BYTES);
           for (int kb = 0; kb < KB; ++kb)
-            tma_load_4d(smem + C::Q_OFF + t * C::TILE_BYTES + kb * 16384, &tm_q, &q_full[t], kb * 64, I.h,
+            tma_load_4d(smem + C::Q_OFF + t * C::TILE_BYTES + kb * 16384, &tm_q, &q_full[t], kb * BOX_COLS, I.h,
                         I.q0 + t * 128, I.b);
           q_loaded |= 1u << t;
           q_par ^= 1u << t;
@@ -220,7 +234,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           mbar_arrive_expect_tx(&kv_full[slot], C::TILE_BYTES);
           const CUtensorMap* m = (i & 1) ? &tm_v : &tm_k;
           uint8_t* dst = smem + C::KV_OFF + slot * C::TILE_BYTES;
-          for (int kb = 0; kb < KB; ++kb) tma_load_4d(dst + kb * 16384, m, &kv_full[slot], kb * 64, I.hkv, (i >> 1) * 128, I.b);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_4d(dst + kb * 16384, m, &kv_full[slot], kb * BOX_COLS, I.hkv, (i >> 1) * 128, I.b);
           ++it;
         }
       }
@@ -232,24 +247,36 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t IDESC_S = FP8 ? idesc_e4m3_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t IDESC_O = FP8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
+      // every instruction consumes 32 bytes of K: 16 bf16 or 32 e4m3 elements
+      constexpr int KS_S = D * C::ES / 32, KS_PV = 128 * C::ES / 32;
       const uint32_t q_base = smem_u32(smem + C::Q_OFF);
       const uint32_t kv_base = smem_u32(smem + C::KV_OFF);
       auto issue_s = [&](int t, int slot) {
         const uint32_t qa = q_base + t * C::TILE_BYTES, ka = kv_base + slot * C::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < KS_S; ++kk) {
           const uint32_t o = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + t * 128, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), IDESC_S, kk > 0);
+          if constexpr (FP8)
+            umma_ss_f8(tmem + t * 128, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), IDESC_S, kk > 0);
+          else
+            umma_ss(tmem + t * 128, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(ka + o, 16, 1024), IDESC_S, kk > 0);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
         const uint32_t va = kv_base + slot * C::TILE_BYTES;
+        // P (K = 128 keys) from TMEM, 8 columns per instruction; V MN-major,
+        // 32 bytes of keys (16 or 32 rows of 128 bytes) per instruction
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), IDESC_O,
-                  (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < KS_PV; ++kk) {
+          if constexpr (FP8)
+            umma_ts_f8(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 4096, 16384, 1024), IDESC_O,
+                       (acc || kk > 0) ? 1u : 0u);
+          else
+            umma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), IDESC_O,
+                    (acc || kk > 0) ? 1u : 0u);
+        }
       };
       auto wait_item = [&](int i) { return mbar_wait(&kv_full[i % NS], (i / NS) & 1, lim, W_FWD_KV_FULL); };
 
@@ -316,7 +343,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   // Take the launch budget back only after the softmax warps have returned
   // theirs (named barrier 2): re-acquiring earlier could starve a softmax warp
   // that has not yet grown, and both would wait forever.
-  asm volatile("bar.sync 2, %0;" :: "n"(FwdCfg<D>::THREADS) : "memory");
+  asm volatile("bar.sync 2, %0;" :: "n"(C::THREADS) : "memory");
   setmaxnreg_inc<FWD_LAUNCH_REGS>();
   } else {
     setmaxnreg_inc<FWD_SOFTMAX_REGS>();
@@ -382,6 +409,46 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             tmem_st_32x32b_x32(t_s + half * 32, pk);
           }
         };
+        if constexpr (FP8) {
+          // tile max first, then P = 2^(s - m + FWD_F8_P_LOG2) as e4m3, four per column
+          float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+  #pragma unroll
+          for (int c = 4; c < 128; c += 4) {
+            mx0 = fmaxf(mx0, s[c]); mx1 = fmaxf(mx1, s[c + 1]); mx2 = fmaxf(mx2, s[c + 2]); mx3 = fmaxf(mx3, s[c + 3]);
+          }
+          const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+          const bool resc = m_tile > m_used + FWD_F8_TAU;   // false while both are -inf
+          float alpha = 1.f;
+          if (resc) { alpha = ex2_approx(m_used - m_tile); l *= alpha; lr *= alpha; m_used = m_tile; }
+          if (j > 0 && __any_sync(0xffffffffu, resc)) {
+  #pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld_32x32b_x32(t_o + c0, ov);
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st_32x32b_x32(t_o + c0, ov);
+            }
+          }
+          const float msub = (m_used == -INFINITY) ? 0.f : m_used - FWD_F8_P_LOG2;
+  #pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = half * 64 + 4 * i;
+              float x0, x1, x2, x3;
+              ffma2(x0, x1, s[c], s[c + 1], sl2, sl2, -msub, -msub);
+              ffma2(x2, x3, s[c + 2], s[c + 3], sl2, sl2, -msub, -msub);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+              pk[i] = pack_e4m3x4(p0, p1, p2, p3);
+              fadd2(ls0, ls1, ls0, ls1, p0, p1);
+              fadd2(ls0, ls1, ls0, ls1, p2, p3);
+              add_e4m3x4_f32(lr0, lr1, pk[i]);
+            }
+            tmem_st_32x32b_x16(t_s + half * 16, pk);
+          }
+        } else {
         bool slow = __any_sync(0xffffffffu, m_used == -INFINITY);
         if (!slow) {
           // the branch keeps the polynomial loop and the all-MUFU loop apart, so
@@ -412,6 +479,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           }
           exp_tile((m_used == -INFINITY) ? 0.f : m_used, false);
         }
+        }
         l += ls0 + ls1;
         lr += lr0 + lr1;
         tmem_st_wait();
@@ -424,9 +492,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       if (nt > 0) ++o_cnt;
       if (have_o) tc_fence_after();
       const bool has = l > 0.f;
-      const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
+      const float inv_l = (lr > 0.f) ? p.o_scale / lr : 0.f;
+      const float m_lse = FP8 ? m_used - FWD_F8_P_LOG2 : m_used;   // the reference l is counted against
       if (row < p.Lq && p.lse != nullptr)
-        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_used + log2f(l)) * LN2 : -INFINITY;
+        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_lse + log2f(l)) * LN2 : -INFINITY;
       const size_t orow = (static_cast<size_t>(b) * p.Lq + row) * p.Hq + h;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -459,7 +528,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       }
     }
     setmaxnreg_dec<FWD_LAUNCH_REGS>();    // give the extra registers back first
-    asm volatile("bar.arrive 2, %0;" :: "n"(FwdCfg<D>::THREADS) : "memory");
+    asm volatile("bar.arrive 2, %0;" :: "n"(C::THREADS) : "memory");
   }
 
   tc_fence_before();

@@ -166,6 +166,20 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
                "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
                :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// kind::f8f6f4 forms (8-bit inputs, here e4m3, fp32 accumulate; K = 32 per instruction).
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+               :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// A in tensor memory: four e4m3 values per 32-bit column, K-major.
+__device__ __forceinline__ void umma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+               :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
 // Arrives once on `bar` when every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -178,6 +192,13 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
          (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32, A and B e4m3 (format code 0),
+// dense; same bit positions as above.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor with the 128-byte swizzle: start address,
@@ -221,6 +242,28 @@ __device__ __forceinline__ void add_bf16x2_f32(float& lo_acc, float& hi_acc, uin
   asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
       "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
       : "+f"(lo_acc), "+f"(hi_acc) : "r"(pk));
+}
+
+// Four floats rounded to e4m3 (nearest, saturating at +-448), packed with v0
+// in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r) : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+  return r;
+}
+// a0 += e4m3 bytes 0 and 2 of pk, a1 += bytes 1 and 3 (exact: e4m3 -> f16 -> f32 adds)
+__device__ __forceinline__ void add_e4m3x4_f32(float& a0, float& a1, uint32_t pk) {
+  asm("{\n\t.reg .b16 lo, hi, h0, h1, h2, h3;\n\t.reg .b32 f01, f23;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 f01, lo;\n\tcvt.rn.f16x2.e4m3x2 f23, hi;\n\t"
+      "mov.b32 {h0, h1}, f01;\n\tmov.b32 {h2, h3}, f23;\n\t"
+      "add.rn.f32.f16 %0, h0, %0;\n\tadd.rn.f32.f16 %1, h1, %1;\n\t"
+      "add.rn.f32.f16 %0, h2, %0;\n\tadd.rn.f32.f16 %1, h3, %1;\n\t}"
+      : "+f"(a0), "+f"(a1) : "r"(pk));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

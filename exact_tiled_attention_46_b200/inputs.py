@@ -23,6 +23,10 @@ then round-to-nearest-even to bf16 through torch):
   fixed-size pages: the pages a sequence needs are drawn, in a seeded random
   order, from ``default_rng([seed, 0, 2])``; unused table entries are -1 and
   spare pool pages hold a fill value;
+* e4m3 (FP8) prefill inputs are the same float32 draws as the bf16 ones,
+  divided by a per-tensor scale (max |x| / 448, e4m3's largest finite value)
+  and rounded to e4m3 (nearest even) through torch; the value of an element is
+  its e4m3 value times the scale;
 * the new token's rows of a decode step with KV append come from
   ``default_rng([seed, 0, 1])`` (K then V, [B, Hkv, D]).
 
@@ -191,3 +195,34 @@ def paged_decode_inputs(B, Hq, Hkv, D, page_size, seed, len_lo, len_hi, lens=Non
             dst.index_copy_(0, idx, full.view(m, page_size, Hkv, D).to(dev))
     return {"q": q, "k_pages": kp, "v_pages": vp, "page_table": torch.from_numpy(table),
             "seqlens": torch.from_numpy(lens.copy())}
+
+
+E4M3_MAX = 448.0
+
+
+def to_e4m3(x: np.ndarray):
+    """(e4m3 tensor, scale) with x ~= e4m3 * scale; scale = max|x| / 448 (1 for all-zero x)."""
+    amax = float(np.max(np.abs(x))) if x.size else 0.0
+    scale = amax / E4M3_MAX if amax > 0 else 1.0
+    t = torch.from_numpy(np.ascontiguousarray(x / np.float32(scale), dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t, scale
+
+
+def dequant_f64(t: torch.Tensor, scale: float) -> np.ndarray:
+    """Exact float64 value of an e4m3 tensor times its scale."""
+    return t.to(torch.float64).numpy() * float(scale)
+
+
+def prefill_inputs_fp8(B, Hq, Hkv, Lq, Lk, D, seed, q_boost_heads=0):
+    """e4m3 Q [B,Lq,Hq,D], K/V [B,Lk,Hkv,D] (CPU tensors) and their scales,
+    from the same draws as ``prefill_inputs``."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Lq, Hq, D), dtype=np.float32)
+    if q_boost_heads:
+        q[:, :, :q_boost_heads, :] *= 4.0
+    k = rng.standard_normal((B, Lk, Hkv, D), dtype=np.float32)
+    v = rng.standard_normal((B, Lk, Hkv, D), dtype=np.float32)
+    out = {}
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        out[name], out[name + "_scale"] = to_e4m3(x)
+    return out

@@ -76,6 +76,24 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float*
                     int o_dtype, fa_stream_t stream);
 
 /*
+ * Prefill forward on e4m3 (FP8) inputs ("FlashAttention Explained ...",
+ * section "FlashAttention-4 and Newer Research": later versions rework
+ * precision among other things).  q, k, v hold one e4m3 byte per element in
+ * the usual layouts; the value of an element is its e4m3 value times the
+ * tensor's scale (q_scale, k_scale, v_scale: finite, > 0).  Both products run
+ * on the tensor cores in e4m3 with fp32 accumulation: S = (q k^T) * q_scale *
+ * k_scale * scale, and P (kept in e4m3, scaled by 2^8 against the running
+ * max) times v.  o (o_dtype) and lse are as in fa_fwd, in the dequantized
+ * units.  The only rounding beyond fa_fwd's is that of P to e4m3 (relative
+ * 2^-4, or 2^-18 of the row's largest probability absolute), which moves O by
+ * at most that much of the spread of the attended v rows; the LSE uses the
+ * unrounded probabilities.  D must be 128 (else FA_ERR_UNSUPPORTED).
+ */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float q_scale, float k_scale,
+                     float v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Lq, int Lk,
+                     int D, float scale, int causal, int o_dtype, fa_stream_t stream);
+
+/*
  * Backward ("FlashAttention Explained ...", section "More Efficient
  * Backpropagation"; "How FlashAttention Speeds Up LLM Attention", "Recompute
  * probabilities for training"): probabilities are recomputed per tile from q,
@@ -241,7 +259,8 @@ fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t strea
  * cached verdict (0 not yet checked, 1 match, 2 mismatch; never changed by
  * this call); *expected_regs, the figure the split assumes; *num_regs, the
  * compiled count (queried from the runtime, which needs a GPU; pass NULL to
- * skip).  D must be 64 or 128.  No counterpart on the pages.
+ * skip).  D must be 64 or 128, or -128 for the e4m3 forward (bwd = 0).  No
+ * counterpart on the pages.
  */
 fa_status fa_launch_guard(int bwd, int D, int causal, int* num_regs, int* expected_regs, int* state);
 

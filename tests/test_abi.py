@@ -198,3 +198,18 @@ def test_decode_paged_rejects_bad_arguments(L):
     a = list(ok)
     a[12] = 0                                              # empty pool
     assert L.fa_decode_paged_splitkv(*a) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fwd_fp8_rejects_bad_arguments(L):
+    # q, k, v, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, Lq, Lk, D, scale, causal, o_dtype, stream
+    ok = [P16, P16, P16, 1.0, 1.0, 1.0, P16, None, 1, 2, 2, 8, 8, 128, 0.1, 1, 0, None]
+    a = list(ok)
+    a[13] = 64
+    assert L.fa_fwd_fp8(*a) == fa.FA_ERR_UNSUPPORTED
+    for i in (3, 4, 5):
+        a = list(ok)
+        a[i] = 0.0                                          # scales must be > 0
+        assert L.fa_fwd_fp8(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[1] = P16 + 8
+    assert L.fa_fwd_fp8(*a) == fa.FA_ERR_INVALID_ARG

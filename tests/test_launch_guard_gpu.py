@@ -34,6 +34,12 @@ def test_every_instantiation_compiles_to_the_split_register_count(bwd, D, causal
     assert regs == expected, f"{'bwd' if bwd else 'fwd'}<{D},{causal}>: {regs} registers, split assumes {expected}"
 
 
+@pytest.mark.parametrize("causal", [0, 1])
+def test_fp8_forward_compiles_to_the_split_register_count(causal):
+    regs, expected, _ = fa.launch_guard(0, -128, causal)
+    assert regs == expected, f"fwd_fp8<{causal}>: {regs} registers, split assumes {expected}"
+
+
 CHILD = r"""
 import torch, exact_tiled_attention_46_b200 as fa
 def states():
