@@ -24,7 +24,7 @@ __all__ = ["fwd", "bwd", "decode", "decode_combine", "device_status", "set_wait_
            "selftest_wait_timeout", "lib", "LIB_PATH", "FA_OK", "FA_ERR_INVALID_ARG",
            "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FaError",
            "bwd_workspace_size", "decode_workspace_size", "decode_chunk", "launch_guard", "decode_append",
-           "decode_paged", "fwd_fp8"]
+           "decode_paged", "fwd_fp8", "attn_merge"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa46.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -43,6 +43,7 @@ _SIGNATURES = {
     "fa_decode_workspace_size": ([_i, _i, _i, _i], _sz),
     "fa_decode_splitkv": ([_vp] * 6 + [_i] * 5 + [_f, _i, _vp, _sz, _vp], _i),
     "fa_decode_combine": ([_vp] * 5 + [_i] * 5 + [_vp], _i),
+    "fa_attn_merge": ([_vp] * 6 + [_i] * 5 + [_vp], _i),
     "fa_decode_append_splitkv": ([_vp] * 8 + [_i] * 5 + [_f, _i, _vp, _sz, _vp], _i),
     "fa_decode_paged_splitkv": ([_vp] * 9 + [_i] * 7 + [_f, _i, _vp, _sz, _vp], _i),
     "fa_decode_splitkv_static": ([_vp] * 6 + [_i] * 5 + [_f, _i, _vp], _i),
@@ -290,6 +291,26 @@ def decode_combine(o_part, lse_part, num_splits=None, o_dtype=torch.bfloat16):
     _check(lib().fa_decode_combine(o_part.data_ptr(), lse_part.data_ptr(), ns_ptr, out.data_ptr(), lse.data_ptr(),
                                    B, Hq, D, S, _odt(o_dtype), _stream(o_part)), "fa_decode_combine")
     return out, lse
+
+
+def attn_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None, o_dtype=torch.float32):
+    """Merge two results over disjoint key sets: o_* [B,L,H,D] fp32, lse_* [B,H,L] -> (o, lse).
+
+    ``out`` / ``lse_out`` may be ``o_a`` / ``lse_a`` (in-place accumulation).
+    """
+    _need(o_a, "o_a", dtype=torch.float32, ndim=4)
+    _need(o_b, "o_b", dtype=torch.float32, ndim=4)
+    _need(lse_a, "lse_a", dtype=torch.float32, ndim=3)
+    _need(lse_b, "lse_b", dtype=torch.float32, ndim=3)
+    B, L, H, D = o_a.shape
+    if out is None:
+        out = torch.empty((B, L, H, D), dtype=o_dtype, device=o_a.device)
+    _need(out, "out", dtype=None, ndim=4)
+    if lse_out is None:
+        lse_out = torch.empty((B, H, L), dtype=torch.float32, device=o_a.device)
+    _check(lib().fa_attn_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(), out.data_ptr(),
+                               lse_out.data_ptr(), B, H, L, D, _odt(out.dtype), _stream(o_a)), "fa_attn_merge")
+    return out, lse_out
 
 
 def device_status(reset: bool = False, device=None):

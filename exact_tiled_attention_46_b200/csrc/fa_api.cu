@@ -430,6 +430,28 @@ fa_status fa_decode_paged_splitkv(const void* q, const void* k_new, const void* 
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_attn_merge(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b, void* o_out,
+                        float* lse_out, int B, int H, int L, int D, int o_dtype, fa_stream_t stream) {
+  if (B <= 0 || H <= 0 || L < 0 || D <= 0 || D % 4 != 0) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_BF16 && o_dtype != FA_FP32) return FA_ERR_INVALID_ARG;
+  if (L == 0) return FA_OK;
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o_out)) return FA_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(lse_a) | reinterpret_cast<uintptr_t>(lse_b) |
+        reinterpret_cast<uintptr_t>(lse_out)) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  // the output may be either input: every element is read by the thread that writes it, before it writes
+  fa::MergeParams p;
+  p.o_a = o_a; p.lse_a = lse_a; p.o_b = o_b; p.lse_b = lse_b; p.o_out = o_out; p.lse_out = lse_out;
+  p.B = B; p.H = H; p.L = L; p.D = D; p.o_fp32 = (o_dtype == FA_FP32);
+  const size_t rows = size_t(B) * L * H;
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 7) / 8, size_t(sms) * 16));
+  fa::attn_merge_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
 fa_status fa_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
                                    void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
                                    int o_dtype, fa_stream_t stream) {

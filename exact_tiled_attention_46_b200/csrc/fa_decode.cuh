@@ -573,4 +573,53 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const CombineParams
   if (threadIdx.x == 0 && p.lse != nullptr) p.lse[bh] = has ? mx + logf(wsum) : -INFINITY;
 }
 
+// Merge of two attention results over disjoint key sets, row by row, in the
+// prefill layout (the merge step of context-parallel prefill: each rank's
+// queries meet the key blocks one at a time):
+//   lse = ln(e^lse_a + e^lse_b),  o = e^(lse_a - lse) o_a + e^(lse_b - lse) o_b,
+// an empty side having lse = -inf.  o_* [B, L, H, D] fp32, lse_* [B, H, L].
+// One warp per (b, l, h) row; o_out / lse_out may be o_a / lse_a.
+struct MergeParams {
+  const float* o_a; const float* lse_a;
+  const float* o_b; const float* lse_b;
+  void* o_out; float* lse_out;
+  int B, H, L, D, o_fp32;
+};
+__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+  const int lane = threadIdx.x & 31;
+  const size_t rows = static_cast<size_t>(p.B) * p.L * p.H;
+  for (size_t row = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; row < rows;
+       row += static_cast<size_t>(gridDim.x) * blockDim.x / 32) {
+    const int h = static_cast<int>(row % p.H);
+    const size_t bl = row / p.H;
+    const int l = static_cast<int>(bl % p.L);
+    const int b = static_cast<int>(bl / p.L);
+    const size_t li = (static_cast<size_t>(b) * p.H + h) * p.L + l;
+    const float la = p.lse_a[li], lb = p.lse_b[li];
+    const float mx = fmaxf(la, lb);
+    const bool empty = mx == -INFINITY;
+    const float wa = (la == -INFINITY) ? 0.f : expf(la - mx);
+    const float wb = (lb == -INFINITY) ? 0.f : expf(lb - mx);
+    const float inv = empty ? 0.f : 1.f / (wa + wb);
+    const float ca = wa * inv, cb = wb * inv;
+    const float* oa = p.o_a + row * p.D;
+    const float* ob = p.o_b + row * p.D;
+    for (int d = lane * 4; d < p.D; d += 128) {
+      const float4 x = *reinterpret_cast<const float4*>(oa + d);
+      const float4 y = *reinterpret_cast<const float4*>(ob + d);
+      const float4 r = make_float4(ca * x.x + cb * y.x, ca * x.y + cb * y.y, ca * x.z + cb * y.z, ca * x.w + cb * y.w);
+      if (p.o_fp32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.o_out) + row * p.D + d) = r;
+      } else {
+        uint2 w;
+        w.x = pack_bf16x2(r.x, r.y);
+        w.y = pack_bf16x2(r.z, r.w);
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.o_out) + row * p.D + d) = w;
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && p.lse_out != nullptr) p.lse_out[li] = empty ? -INFINITY : mx + logf(wa + wb);
+  }
+}
+
 }  // namespace fa

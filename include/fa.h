@@ -226,6 +226,24 @@ fa_status fa_decode_combine(const float* o_part, const float* lse_part, const in
                             int o_dtype, fa_stream_t stream);
 
 /*
+ * Merge of two attention results over disjoint key sets, in the prefill
+ * layout: the step that joins the partial results of context-parallel (ring)
+ * prefill, where a rank's queries meet the key/value blocks one at a time
+ * ("How FlashAttention Speeds Up LLM Attention": partial results kept on a
+ * common numerical scale are combined; "FlashAttention Explained ...",
+ * "Longer Context Windows").  o_a, o_b [B,L,H,D] fp32 are normalised outputs
+ * over the two key sets, lse_a, lse_b [B,H,L] fp32 their natural
+ * log-sum-exps (-inf for a row with no key in that set).  Writes
+ *   lse_out = ln(e^lse_a + e^lse_b),  o_out = e^(lse_a - lse_out) o_a + e^(lse_b - lse_out) o_b
+ * (o_out in o_dtype; a row empty on both sides gets 0 and -inf).  o_out may
+ * be o_a or o_b (fp32) and lse_out lse_a or lse_b (in-place accumulation);
+ * lse_out may be NULL.  D must be a multiple of 4.
+ */
+fa_status fa_attn_merge(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b,
+                        void* o_out, float* lse_out, int B, int H, int L, int D, int o_dtype,
+                        fa_stream_t stream);
+
+/*
  * Device status of the current device: *code receives 0 (ok), FA_ERR_TIMEOUT
  * when some kernel's bounded wait ran out since the last reset, or
  * FA_ERR_INVALID_ARG when a kernel met device-side input it could not honour

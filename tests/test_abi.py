@@ -213,3 +213,20 @@ def test_fwd_fp8_rejects_bad_arguments(L):
     a = list(ok)
     a[1] = P16 + 8
     assert L.fa_fwd_fp8(*a) == fa.FA_ERR_INVALID_ARG
+
+
+def test_attn_merge_rejects_bad_arguments(L):
+    # o_a, lse_a, o_b, lse_b, o_out, lse_out, B, H, L, D, o_dtype, stream
+    ok = [P16] * 6 + [1, 2, 8, 128, 1, None]
+    a = list(ok)
+    a[9] = 126                                             # D not a multiple of 4
+    assert L.fa_attn_merge(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[2] = None
+    assert L.fa_attn_merge(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[1] = P16 + 2
+    assert L.fa_attn_merge(*a) == fa.FA_ERR_INVALID_ARG
+    a = list(ok)
+    a[8] = 0                                               # nothing to merge
+    assert L.fa_attn_merge(*a) == fa.FA_OK
