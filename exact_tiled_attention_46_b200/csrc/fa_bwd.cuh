@@ -22,6 +22,8 @@
 //        warps 0-7  one thread per key row; warps w and w + 4 share a TMEM lane
 //                   quadrant and take 64 of the 128 query columns each (no row
 //                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
+//                   on the tiles that need it; P^T is published first (the dV
+//                   products run while dS^T is formed from P read back)
 //        warps 8-11 one thread per query row: dQ tile from TMEM (two buffers at
 //                   D = 64) into a swizzled shared-memory box per warp, added to
 //                   the fp32 accumulator by TMA reduce-add (32 rows x 32
@@ -318,38 +320,77 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int cmin = key < p.Lk ? (CAUSAL ? key - off - i * 128 : -1) : (1 << 30);
       const int rowoff = r * 128;
       bool ok = true;
+      // Phase 1: P^T = 2^(S^T * scale - LSE) (masked), as P_hi + P_lo over the
+      // S^T columns it comes from; published at once, so that the dV products
+      // run while phase 2 forms dS^T.
 #pragma unroll
       for (int lc = 0; lc < 2; ++lc) {
         const int c0 = hh * 64 + lc * 32;              // first query column of this chunk
-        uint32_t sv[32], dp[32];
+        uint32_t sv[32];
         tmem_ld_32x32b_x32(tmem + lane_bits + C::T_S + c0, sv);
-        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_DP + c0, dp);
-        uint32_t phi[16], plo[16], dhi[16], dlo[16];
+        // the mask only matters where some key row of the warp starts after c0
+        // (the causal diagonal, keys past Lk); elsewhere every column is allowed
+        const bool masked = __any_sync(0xffffffffu, cmin > c0);
+        uint32_t phi[16], plo[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int c = c0 + 2 * t;
-          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + c);
-          const float2 d2 = *reinterpret_cast<const float2*>(dlt + c);
-          float x0, x1;
-          ffma2(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), sl2, sl2, -l2.x, -l2.y);
-          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          p0 = (c >= cmin) ? p0 : 0.f;
-          p1 = (c + 1 >= cmin) ? p1 : 0.f;
-          phi[t] = pack_bf16x2(p0, p1);
-          float r0, r1;
-          fadd2(r0, r1, p0, p1, -__uint_as_float(phi[t] << 16), -__uint_as_float(phi[t] & 0xffff0000u));
-          plo[t] = pack_bf16x2(r0, r1);
-          float e0, e1, s0, s1;
-          fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -d2.x, -d2.y);
-          ffma2(s0, s1, p0, p1, e0, e1, 0.f, 0.f);
-          dhi[t] = pack_bf16x2(s0, s1);
-          fadd2(r0, r1, s0, s1, -__uint_as_float(dhi[t] << 16), -__uint_as_float(dhi[t] & 0xffff0000u));
-          dlo[t] = pack_bf16x2(r0, r1);
+        for (int t4 = 0; t4 < 8; ++t4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + 4 * t4);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = 2 * t4 + u;
+            const int c = c0 + 2 * t;
+            float x0, x1;
+            ffma2(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), sl2, sl2,
+                  -(u ? l4.z : l4.x), -(u ? l4.w : l4.y));
+            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if (masked) {
+              p0 = (c >= cmin) ? p0 : 0.f;
+              p1 = (c + 1 >= cmin) ? p1 : 0.f;
+            }
+            phi[t] = pack_bf16x2(p0, p1);
+            float r0, r1;
+            resid_bf16x2(phi[t], p0, p1, r0, r1);
+            plo[t] = pack_bf16x2(r0, r1);
+          }
         }
         // P_hi and P_lo of query columns [c0, c0+32) go back over the 32 S^T columns
         // just read: P_hi to the first 16, P_lo to the next 16
         tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + c0, phi);
         tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + c0 + 16, plo);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      // Phase 2: dS^T = P^T * (dP^T - Delta), P^T = P_hi + P_lo read back, as
+      // dS_hi + dS_lo into swizzled shared memory.
+#pragma unroll
+      for (int lc = 0; lc < 2; ++lc) {
+        const int c0 = hh * 64 + lc * 32;
+        uint32_t dp[32], ph[16], pl[16];
+        tmem_ld_32x32b_x32_nowait(tmem + lane_bits + C::T_DP + c0, dp);
+        tmem_ld_32x32b_x16_nowait(tmem + lane_bits + C::T_S + c0, ph);
+        tmem_ld_32x32b_x16_nowait(tmem + lane_bits + C::T_S + c0 + 16, pl);
+        tmem_ld_wait_regs(dp);
+        tmem_ld_wait_regs(ph);
+        tmem_ld_wait_regs(pl);
+        uint32_t dhi[16], dlo[16];
+#pragma unroll
+        for (int t4 = 0; t4 < 8; ++t4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dlt + c0 + 4 * t4);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = 2 * t4 + u;
+            float p0 = __uint_as_float(pl[t] << 16), p1 = __uint_as_float(pl[t] & 0xffff0000u);
+            add_bf16x2_f32(p0, p1, ph[t]);
+            float e0, e1, s0, s1, r0, r1;
+            fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -(u ? d4.z : d4.x),
+                  -(u ? d4.w : d4.y));
+            ffma2(s0, s1, p0, p1, e0, e1, 0.f, 0.f);
+            dhi[t] = pack_bf16x2(s0, s1);
+            resid_bf16x2(dhi[t], s0, s1, r0, r1);
+            dlo[t] = pack_bf16x2(r0, r1);
+          }
+        }
         // the shared-memory operands of pair n - 1 must have been consumed
         if (lc == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
         // columns c0..c0+31: 4 16-byte chunks of the 128-byte row of block hh (128B swizzle)
@@ -362,10 +403,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       if (!ok) break;
-      tmem_st_wait();
       fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_ready);
+      tc_fence_before();                               // the phase-2 reads of P and dP^T come first
       mbar_arrive(ds_ready);
     }
     setmaxnreg_dec<BWD_LAUNCH_REGS>();
