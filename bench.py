@@ -1,6 +1,6 @@
 """Benchmark of the exact tiled attention kernels on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick] [--config 1-5]
 
 Headline (one JSON line on rank 0): causal bf16 prefill forward on
 B=4, Hq=Hkv=16, L=2048, D=128 (Q x4 on heads 0-7, seed 1), in TFLOP/s with the
@@ -619,6 +619,43 @@ def run_profile_case(args):
     print(f"profile case {name}: {args.warmup + args.steps} launches done")
 
 
+CONFIGS = {1: "tiny_fwd", 2: "causal_prefill", 3: "long_gqa_prefill", 4: "train_fwd_bwd", 5: "splitkv_decode"}
+
+
+def run_config(args):
+    """One workload alone (configs 1-5 in the order the workloads are listed);
+    prints one JSON line with that workload's own metric as the value."""
+    import exact_tiled_attention_46_b200 as fa
+    from exact_tiled_attention_46_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush = l2_flusher(dev)
+    name = CONFIGS[args.config]
+    clocks = ClockSampler(0)
+    clocks.start()
+    if name == "train_fwd_bwd":
+        sec = section_train(fa, args.steps, args.warmup, flush, stream, peaks, peak_src, dev)
+        value, unit, ms = sec.get("tflops_bwd"), "TFLOP/s", sec.get("ms_bwd")
+    elif name == "splitkv_decode":
+        sec, _ = section_decode(fa, args.steps, args.warmup, flush, stream, peaks, peak_src, dev)
+        value, unit, ms = sec["gbs"], "GB/s", sec["ms"]
+    else:
+        sec = section_fwd(fa, name, args.steps, args.warmup, flush, stream, peaks, peak_src, dev)
+        value, unit, ms = sec["tflops"], "TFLOP/s", sec["ms"]
+    ck = clocks.stop()
+    w = synth.WORKLOADS[name]
+    print(json.dumps({"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+                      "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), bf16 RNE)",
+                      "config": {"workload": name, "config_index": args.config, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                                 "L": w.Lk, "D": w.D, "causal": w.causal,
+                                 "l2": "flushed (256 MiB write) before every timed step"},
+                      "roofline": sec.get("roofline"), "clocks": ck, "section": sec}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-case", default=None,
@@ -630,11 +667,16 @@ def main():
     ap.add_argument("--quick", action="store_true", help="headline only, no extra sections")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--config", type=int, choices=sorted(CONFIGS), default=None,
+                    help="time one workload alone (1 tiny, 2 causal prefill = the default headline run, "
+                         "3 long GQA, 4 training backward, 5 decode)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.profile_case:
         run_profile_case(args)
+    elif args.config is not None and args.config != 2 and args.impl == "ours":
+        run_config(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -26,13 +26,17 @@ __all__ = ["fwd", "bwd", "decode", "decode_combine", "device_status", "set_wait_
            "bwd_workspace_size", "decode_workspace_size", "decode_chunk", "launch_guard", "decode_append",
            "decode_paged", "fwd_fp8", "attn_merge"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa46.so")
+# FA46_LIBRARY may name another build of the same library (the debug build,
+# libfa46_debug.so); there is no fallback when it is missing.
+LIB_PATH = os.environ.get("FA46_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa46.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+FA_ERR_DEVICE_INDEX = 5
 FA_BF16, FA_FP32 = 0, 1
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _SIGNATURES = {
     "fa_abi_version": ([], _i),
+    "fa_debug_build": ([], _i),
     "fa_status_string": ([_i], ctypes.c_char_p),
     "fa_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp], _i),

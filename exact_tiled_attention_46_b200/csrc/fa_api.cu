@@ -282,6 +282,14 @@ extern "C" {
 
 int fa_abi_version(void) { return kAbiVersion; }
 
+int fa_debug_build(void) {
+#ifdef FA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 const char* fa_status_string(int s) {
   switch (s) {
     case FA_OK: return "ok";
@@ -289,6 +297,7 @@ const char* fa_status_string(int s) {
     case FA_ERR_UNSUPPORTED: return "unsupported configuration";
     case FA_ERR_CUDA: return "CUDA call failed";
     case FA_ERR_TIMEOUT: return "kernel wait timed out";
+    case FA_ERR_DEVICE_INDEX: return "device index check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -548,7 +557,11 @@ fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream)
       cudaMemcpyFromSymbolAsync(&w, fa::g_fa_dev_where, 4, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (code) *code = (s == fa::FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : (s == fa::FA_DEV_BAD_INPUT) ? FA_ERR_INVALID_ARG : FA_OK;
+  if (code)
+    *code = (s == fa::FA_DEV_TIMEOUT)     ? FA_ERR_TIMEOUT
+            : (s == fa::FA_DEV_BAD_INPUT) ? FA_ERR_INVALID_ARG
+            : (s == fa::FA_DEV_BAD_INDEX) ? FA_ERR_DEVICE_INDEX
+                                          : FA_OK;
   if (where) *where = static_cast<int>(w);
   if (reset) {
     const uint32_t zero = 0;

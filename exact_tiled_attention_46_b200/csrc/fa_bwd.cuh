@@ -469,6 +469,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int t = 0; t < 32; ++t) v[t] = 0u;
         }
         if (key >= p.Lk) continue;
+        if (!index_ok(krow + c0, 32, static_cast<size_t>(p.B) * p.Lk * p.Hkv * D, W_IDX_BWD_DKV)) continue;
         if (p.g_fp32) {
           float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(out) + krow + c0);
 #pragma unroll

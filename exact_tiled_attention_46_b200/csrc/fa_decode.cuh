@@ -496,6 +496,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         O = fmaf(src[2 + d], a, O);
       }
       const size_t prow = (static_cast<size_t>(b) * p.Hq + hq0 + g) * p.max_splits + I.split;
+      if (!index_ok(prow, 1, static_cast<size_t>(p.B) * p.Hq * p.max_splits, W_IDX_DEC_PART)) continue;
       p.o_part[prow * D + d] = L > 0.f ? O / L : 0.f;
       if (d == 0) p.lse_part[prow] = L > 0.f ? (mx + log2f(L)) * LN2 : -INFINITY;
     }
@@ -513,7 +514,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       } else {
         rowaddr = ((static_cast<size_t>(b) * p.cap + I.cached) * p.Hkv + I.hkv) * D;
       }
-      if (room) {
+      const size_t cache_elems = PAGED ? static_cast<size_t>(p.num_pages) * p.page_size * p.Hkv * D
+                                       : static_cast<size_t>(p.B) * p.cap * p.Hkv * D;
+      if (room && index_ok(rowaddr, D, cache_elems, W_IDX_DEC_APPEND)) {
         const int half = lane / (D / 8), c = lane % (D / 8);
         const size_t nrow = (static_cast<size_t>(b) * p.Hkv + I.hkv) * D;
         const uint4 val = reinterpret_cast<const uint4*>((half ? p.v_new : p.k_new) + nrow)[c];
@@ -567,6 +570,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const CombineParams
       acc = fmaf(w, p.o_part[(static_cast<size_t>(bh) * p.max_splits + s) * p.D + d], acc);
     }
     const float v = has ? acc / wsum : 0.f;
+    if (!index_ok(static_cast<size_t>(bh) * p.D + d, 1, static_cast<size_t>(p.B) * p.Hq * p.D, W_IDX_DEC_OUT)) continue;
     if (p.o_fp32) static_cast<float*>(p.o)[static_cast<size_t>(bh) * p.D + d] = v;
     else static_cast<__nv_bfloat16*>(p.o)[static_cast<size_t>(bh) * p.D + d] = __float2bfloat16_rn(v);
   }
@@ -602,6 +606,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
     const float wb = (lb == -INFINITY) ? 0.f : expf(lb - mx);
     const float inv = empty ? 0.f : 1.f / (wa + wb);
     const float ca = wa * inv, cb = wb * inv;
+    if (!index_ok(row * p.D, p.D, rows * p.D, W_IDX_MERGE)) continue;
     const float* oa = p.o_a + row * p.D;
     const float* ob = p.o_b + row * p.D;
     for (int d = lane * 4; d < p.D; d += 128) {

@@ -494,8 +494,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       const bool has = l > 0.f;
       const float inv_l = (lr > 0.f) ? p.o_scale / lr : 0.f;
       const float m_lse = FP8 ? m_used - FWD_F8_P_LOG2 : m_used;   // the reference l is counted against
-      if (row < p.Lq && p.lse != nullptr)
-        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + row] = has ? (m_lse + log2f(l)) * LN2 : -INFINITY;
+      if (row < p.Lq && p.lse != nullptr) {
+        const size_t li = (static_cast<size_t>(b) * p.Hq + h) * p.Lq + row;
+        if (index_ok(li, 1, static_cast<size_t>(p.B) * p.Hq * p.Lq, W_IDX_FWD_LSE))
+          p.lse[li] = has ? (m_lse + log2f(l)) * LN2 : -INFINITY;
+      }
       const size_t orow = (static_cast<size_t>(b) * p.Lq + row) * p.Hq + h;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -507,6 +510,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
         }
         if (row >= p.Lq) continue;
+        if (!index_ok(orow * D + c0, 32, static_cast<size_t>(p.B) * p.Lq * p.Hq * D, W_IDX_FWD_O)) continue;
         if (p.o_fp32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c0);
 #pragma unroll

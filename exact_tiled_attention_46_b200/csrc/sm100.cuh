@@ -16,7 +16,10 @@ namespace fa {
 // A kernel that meets an input it cannot honour (a page index outside the
 // page pool, a sequence with no room for an appended row) stores
 // FA_DEV_BAD_INPUT the same way, skips that work and carries on.
-enum : uint32_t { FA_DEV_OK = 0u, FA_DEV_TIMEOUT = 1u, FA_DEV_BAD_INPUT = 2u };
+// In a build with FA_DEBUG defined, the kernels also check the index of every
+// global store against the size of its tensor; a store that would fall outside
+// stores FA_DEV_BAD_INDEX (with a code naming the store) and is skipped.
+enum : uint32_t { FA_DEV_OK = 0u, FA_DEV_TIMEOUT = 1u, FA_DEV_BAD_INPUT = 2u, FA_DEV_BAD_INDEX = 3u };
 // (the library is one translation unit, so the words are defined here)
 __device__ uint32_t g_fa_dev_status = 0;
 __device__ uint32_t g_fa_dev_where = 0;
@@ -26,6 +29,26 @@ __device__ __forceinline__ void record_status(uint32_t code, uint32_t where) {
     atomicExch(&g_fa_dev_where, where);
 }
 __device__ __forceinline__ void record_timeout(uint32_t where) { record_status(FA_DEV_TIMEOUT, where); }
+
+// Debug-build index check: true when the element range [first, first + n) lies
+// inside a tensor of `size` elements; otherwise records FA_DEV_BAD_INDEX and
+// returns false, so that the caller skips the access.  Always true (and free)
+// in the normal build.
+__device__ __forceinline__ bool index_ok(size_t first, size_t n, size_t size, uint32_t where) {
+#ifdef FA_DEBUG
+  if (first + n > size) {
+    record_status(FA_DEV_BAD_INDEX, where);
+    return false;
+  }
+#else
+  (void)first; (void)n; (void)size; (void)where;
+#endif
+  return true;
+}
+enum : uint32_t {
+  W_IDX_FWD_O = 0x401, W_IDX_FWD_LSE = 0x402, W_IDX_DEC_PART = 0x403, W_IDX_DEC_APPEND = 0x404,
+  W_IDX_DEC_OUT = 0x405, W_IDX_BWD_DKV = 0x406, W_IDX_MERGE = 0x407
+};
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -50,7 +50,8 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, workspace too small */
   FA_ERR_UNSUPPORTED = 2, /* valid but not implemented here (e.g. D not in {64,128}) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, tensor map) */
-  FA_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fa_device_status) */
+  FA_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (see fa_device_status) */
+  FA_ERR_DEVICE_INDEX = 5 /* debug build: a kernel's store index check failed (see fa_device_status) */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP32 = 1 } fa_dtype;
@@ -60,6 +61,15 @@ int fa_abi_version(void);
 
 /* Static text for a status code; never NULL. */
 const char* fa_status_string(int status);
+
+/*
+ * 1 for the debug build (compiled with FA_DEBUG: every global store of every
+ * kernel checks its index against the size of its tensor; an out-of-range
+ * store is skipped and fa_device_status() reports FA_ERR_DEVICE_INDEX), else
+ * 0.  The debug build is libfa46_debug.so beside libfa46.so; no counterpart
+ * on the pages.
+ */
+int fa_debug_build(void);
 
 /*
  * Prefill forward.  Reads q, k, v (bf16); writes o (bf16) and, when lse is
@@ -248,8 +258,9 @@ fa_status fa_attn_merge(const float* o_a, const float* lse_a, const float* o_b, 
  * when some kernel's bounded wait ran out since the last reset, or
  * FA_ERR_INVALID_ARG when a kernel met device-side input it could not honour
  * (a page index outside the pool, a sequence without room for an appended
- * row) and skipped that work; *where a code naming the place (first event
- * since the reset wins).  Synchronises `stream`.  reset != 0 clears the status.
+ * row) and skipped that work, or FA_ERR_DEVICE_INDEX when, in the debug
+ * build, a store failed its index check; *where a code naming the place (first
+ * event since the reset wins).  Synchronises `stream`.  reset != 0 clears the status.
  */
 fa_status fa_device_status(int* code, int* where, int reset, fa_stream_t stream);
 

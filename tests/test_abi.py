@@ -33,8 +33,8 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_abi_version_and_strings(L):
     assert L.fa_abi_version() == 1
-    for code in range(5):
-        assert L.fa_status_string(code)
+    for code in range(6):
+        assert L.fa_status_string(code) and L.fa_status_string(code) != b"unknown status"
     assert L.fa_status_string(99) == b"unknown status"
 
 
@@ -230,3 +230,15 @@ def test_attn_merge_rejects_bad_arguments(L):
     a = list(ok)
     a[8] = 0                                               # nothing to merge
     assert L.fa_attn_merge(*a) == fa.FA_OK
+
+
+def test_debug_build_compiles_exports_and_reports_itself(L):
+    """The FA_DEBUG build (index checks on every global store) builds from the
+    same sources, exports the same symbols and says which build it is."""
+    path = fabuild.build(debug=True)
+    D = ctypes.CDLL(path)
+    for n in declared_symbols():
+        assert hasattr(D, n), n
+    D.fa_status_string.restype = ctypes.c_char_p
+    assert D.fa_debug_build() == 1 and L.fa_debug_build() == 0
+    assert D.fa_status_string(fa.FA_ERR_DEVICE_INDEX) == b"device index check failed (debug build)"
