@@ -56,12 +56,20 @@ PROFILED_TRAFFIC = {
     "fwd_kernel long_gqa_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
                                     "sha256_16": "88f18afadce39b9c", "bytes": 340705024 + 98593280},
     "bwd_main_kernel train_fwd_bwd": {"sources": ("csrc/fa_bwd.cuh", "csrc/sm100.cuh"),
-                                      "sha256_16": "524f18781031d1ce", "bytes": 407153920 + 225418496},
-    # captured on the first 16 sequences of the decode workload (1.359 GB of KV
-    # rows): 1.36014 GB read + 8.544 MB written, scaled by the KV bytes of a launch
+                                      "sha256_16": "3625827544788fa1", "bytes": 406916864 + 225205760},
+    "fwd_kernel<fp8> causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
+                                       "sha256_16": "ff576a2b73270a40", "bytes": 50417920 + 2505984},
+    # captured on the first 16 sequences of the decode workload (1.35888 GB of KV
+    # rows), scaled to a launch by the KV bytes it reads
     "decode_split_kernel splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
-                                           "sha256_16": "130bae183ee39678",
-                                           "bytes_per_kv_byte": (1360140032 + 8544000) / 1358876672},
+                                           "sha256_16": "475ed25160e6b429",
+                                           "bytes_per_kv_byte": (1360300288 + 8381952) / 1358876672},
+    "decode_split_kernel<append> splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
+                                                   "sha256_16": "475ed25160e6b429",
+                                                   "bytes_per_kv_byte": (1360314624 + 9055488) / 1358876672},
+    "decode_split_kernel<paged16> splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
+                                                    "sha256_16": "475ed25160e6b429",
+                                                    "bytes_per_kv_byte": (1359829248 + 8537088) / 1358876672},
 }
 
 
@@ -256,7 +264,7 @@ def section_fwd_fp8(fa, name, steps, warmup, flush, stream, peaks, peak_src, dev
     tf = fwd_flops(w) / t / 1e12
     fp8_peaks = dict(peaks)
     fp8_peaks["bf16_tflops"] = 2.0 * peaks["bf16_tflops"]
-    r = roofline("tensor", tf, fp8_peaks, peak_src, "TFLOP/s", traffic=None,
+    r = roofline("tensor", tf, fp8_peaks, peak_src, "TFLOP/s", traffic=profiled_traffic(f"fwd_kernel<fp8> {name}"),
                  algorithmic_bytes=fwd_bytes(w) - (w.B * w.Lq * w.Hq * w.D + 2 * w.B * w.Lk * w.Hkv * w.D))
     r["peak_source"] = f"{peak_src} bf16 burst x 2 (nominal fp8:bf16 ratio)"
     r["peak_nominal"] = 2.0 * NOMINAL_PEAKS["bf16_tflops"]
@@ -333,7 +341,8 @@ def section_decode(fa, steps, warmup, flush, stream, peaks, peak_src, dev):
     app = {"workload": "splitkv_decode_append", "kernel": "decode_split_kernel<append>+decode_combine_kernel",
            "ms": ta * 1e3, "ms_median": statistics.median(ms_a), "bytes": kv_bytes + new_bytes, "gbs": gbs_a,
            "frac_hbm": gbs_a / peaks["hbm_gbs"], "launches": 2 * steps,
-           "roofline": roofline("hbm", gbs_a, peaks, peak_src, "GB/s", traffic=None,
+           "roofline": roofline("hbm", gbs_a, peaks, peak_src, "GB/s",
+                                traffic=profiled_traffic("decode_split_kernel<append> splitkv_decode", kv_bytes),
                                 algorithmic_bytes=kv_bytes + new_bytes)}
     return res, app
 
@@ -359,7 +368,10 @@ def section_decode_paged(fa, steps, warmup, flush, stream, peaks, peak_src, dev,
             "kernel": "decode_split_kernel<paged>+decode_combine_kernel", "page_size": page_size,
             "pool_pages": int(kp.shape[0]), "ms": t * 1e3, "ms_median": statistics.median(ms), "kv_bytes": kv_bytes,
             "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "launches": 2 * steps,
-            "roofline": roofline("hbm", gbs, peaks, peak_src, "GB/s", traffic=None, algorithmic_bytes=kv_bytes)}
+            "roofline": roofline("hbm", gbs, peaks, peak_src, "GB/s",
+                                 traffic=profiled_traffic(f"decode_split_kernel<paged{page_size}> splitkv_decode",
+                                                          kv_bytes),
+                                 algorithmic_bytes=kv_bytes)}
 
 
 def run_ours(args):
@@ -588,21 +600,40 @@ def run_profile_case(args):
     """A few launches of one kernel on one workload, for ncu captures (no timing).
 
     causal_prefill / long_gqa_prefill / train_fwd_bwd: fa_fwd (and fa_bwd);
-    splitkv_decode_small: split-KV decode on the first 16 sequences of the
-    decode workload (cache 2.1 GB, larger than L2).
+    splitkv_decode_small / _append_small / _paged16_small: split-KV decode
+    (plain, with the new token appended, from 16-row pages) on the first 16
+    sequences of the decode workload (KV rows 1.36 GB, larger than L2);
+    causal_prefill_fp8: the causal prefill draws quantized to e4m3.
     """
     import exact_tiled_attention_46_b200 as fa
     from exact_tiled_attention_46_b200 import build
     build.build()
     dev = torch.device("cuda", 0)
     name = args.profile_case
-    if name == "splitkv_decode_small":
+    if name in ("splitkv_decode_small", "splitkv_decode_append_small"):
         w = synth.WORKLOADS["splitkv_decode"]
         B = 16
         x = synth.decode_inputs(B, w.Hq, w.Hkv, w.Lk, w.D, w.seed, w.len_lo, w.len_hi, device=dev)
         q, sl = x["q"].to(dev), x["seqlens"].to(dev)
+        kn, vn = (t.to(dev) for t in synth.decode_new_rows(B, w.Hkv, w.D, w.seed))
         for _ in range(args.warmup + args.steps):
-            fa.decode(q, x["k_cache"], x["v_cache"], sl, scale=w.scale)
+            if name == "splitkv_decode_small":
+                fa.decode(q, x["k_cache"], x["v_cache"], sl, scale=w.scale)
+            else:
+                fa.decode_append(q, kn, vn, x["k_cache"], x["v_cache"], sl, scale=w.scale)
+    elif name == "splitkv_decode_paged16_small":
+        w = synth.WORKLOADS["splitkv_decode"]
+        B = 16
+        x = synth.paged_decode_inputs(B, w.Hq, w.Hkv, w.D, 16, w.seed, w.len_lo, w.len_hi, device=dev)
+        q, tab, sl = x["q"].to(dev), x["page_table"].to(dev), x["seqlens"].to(dev)
+        for _ in range(args.warmup + args.steps):
+            fa.decode_paged(q, x["k_pages"], x["v_pages"], tab, sl, scale=w.scale)
+    elif name == "causal_prefill_fp8":
+        w = synth.WORKLOADS["causal_prefill"]
+        x = synth.prefill_inputs_fp8(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.D, w.seed, q_boost_heads=w.q_boost_heads)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        for _ in range(args.warmup + args.steps):
+            fa.fwd_fp8(q, k, v, x["q_scale"], x["k_scale"], x["v_scale"], scale=w.scale, causal=True)
     else:
         w = synth.WORKLOADS[name]
         x = synth.workload_inputs(w)
@@ -659,7 +690,8 @@ def run_config(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-case", default=None,
-                    choices=["causal_prefill", "long_gqa_prefill", "train_fwd_bwd", "splitkv_decode_small"])
+                    choices=["causal_prefill", "long_gqa_prefill", "train_fwd_bwd", "splitkv_decode_small",
+                             "splitkv_decode_append_small", "splitkv_decode_paged16_small", "causal_prefill_fp8"])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
