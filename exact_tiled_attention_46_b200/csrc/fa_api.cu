@@ -217,8 +217,9 @@ fa_status run_decode(const void* q, const void* k_new, const void* v_new, const 
   if (workspace_bytes < fa_decode_workspace_size(B, Hq, static_cast<int>(keys), D)) return FA_ERR_INVALID_ARG;
   const int sub_rows = (page_size % 32 == 0 || !paged) ? 32 : 16;
   CUtensorMap mk, mv;
-  if (!map_bshd(&mk, k_cache, num_pages, page_size, Hkv, D, D, sub_rows, false) ||
-      !map_bshd(&mv, v_cache, num_pages, page_size, Hkv, D, D, sub_rows, false))
+  // boxes of 64 dimensions (128 bytes, 128-byte swizzle) by sub_rows rows
+  if (!map_bshd(&mk, k_cache, num_pages, page_size, Hkv, D, 64, sub_rows, true) ||
+      !map_bshd(&mv, v_cache, num_pages, page_size, Hkv, D, 64, sub_rows, true))
     return FA_ERR_CUDA;
   float* o_part = static_cast<float*>(workspace);
   const size_t lse_off = align_up(size_t(B) * Hq * max_splits * D * 4, 256);

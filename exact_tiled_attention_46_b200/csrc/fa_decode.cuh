@@ -20,12 +20,15 @@
 // Warp NW (the producer) streams K and V tiles of T keys by TMA through an
 // NS-slot mbarrier ring; the rows come from a contiguous cache [B, Lmax, Hkv,
 // D] or, in the PAGED variant, from a page pool [num_pages, page_size, Hkv, D]
-// through a per-sequence page table (one TMA box per page-aligned run of
-// sub_rows rows).  Warps 0..NW-1 split every tile's keys, LPK = D/8 lanes per
-// key, each lane owning 8 consecutive dimensions (one 16-byte chunk of a row).
-// Each key group keeps its own running max / running sum / accumulator (log2
-// units); at the end of the item the groups and warps are merged and the
-// item's normalised partial output and LSE are written.  In the APPEND variant
+// through a per-sequence page table (TMA boxes of 64 dimensions by sub_rows
+// rows, 128-byte swizzled).  Each consumer warp takes 8 of every tile's 32
+// keys: the scores of the GP query heads (padded to 16 rows) come from
+// mma.sync m16n8k16 with K read by ldmatrix, the softmax runs on the score
+// fragments, and P.V is mma.sync m16n8k8 with P straight from the score
+// fragment and V read by ldmatrix.trans, into a 16 x D fp32 accumulator
+// fragment.  Each warp keeps its own running max / sums (log2 units); at the
+// end of the item the warps are merged and the item's normalised partial
+// output and LSE are written.  In the APPEND variant
 // the new token's K and V rows (k_new, v_new) are attended as key seqlens[b]
 // straight from their input rows and written into the cache at row
 // seqlens[b] by one CTA, in the same launch.  The combine kernel merges the
@@ -59,19 +62,19 @@ template <int D, int GP>
 struct DecCfg {
   static constexpr int T = 32;                  // keys per ring slot
   static constexpr int NS = 4;                  // ring slots (K and V tile each)
-  static constexpr int NW = 4;                  // consumer warps
-  static constexpr int LPK = D / 8;             // lanes per key (8 dimensions each)
-  static constexpr int KPW = 32 / LPK;          // keys per warp step
-  static constexpr int TILE_BYTES = T * D * 2;
+  static constexpr int NW = 4;                  // consumer warps, 8 keys of each tile apiece
+  static constexpr int TILE_BYTES = T * D * 2;  // D / 64 blocks of T rows x 128 bytes (128B swizzle)
+  static constexpr int BLOCK_BYTES = T * 128;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int MRG_FLOATS = NW * GP * (D + 2);
+  static constexpr int MRG_STRIDE = D + 4;      // per (warp, head): m, l, l of the rounded p, pad, O[D]
+  static constexpr int MRG_FLOATS = NW * GP * MRG_STRIDE;
   static constexpr int NI = 2;                  // item queue entries (producer -> consumers)
   static constexpr int ITEM_OFF = NS * STAGE_BYTES + MRG_FLOATS * 4;
   static constexpr int BAR_OFF = ITEM_OFF + 16;
-  static constexpr int SMEM_BYTES = BAR_OFF + (2 * NS + 2 * NI) * 8 + 128;
+  static constexpr int SMEM_BYTES = BAR_OFF + (2 * NS + 2 * NI) * 8 + 1024;
   static constexpr int THREADS = (NW + 1) * 32;
   static constexpr int CTAS_PER_SM = 3;
-  static_assert((T / NW) % KPW == 0, "keys per warp must be a multiple of keys per step");
+  static_assert(T == 8 * NW && GP <= 8 && D % 64 == 0, "8 keys per consumer warp; heads fit the 16-row fragment");
 };
 
 constexpr float DEC_TAU = 8.0f;
@@ -80,13 +83,6 @@ enum : uint32_t {
   W_DEC_FULL = 0x201, W_DEC_EMPTY = 0x202, W_DEC_DRAIN = 0x203, W_DEC_PAGE = 0x204, W_DEC_APPEND_ROOM = 0x205,
   W_DEC_APPEND_PAGE = 0x206, W_DEC_ITEM = 0x207, W_DEC_ITEM_EMPTY = 0x208
 };
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {
-  f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
-  f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
-  f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
-  f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
-}
 
 // Keys attended for sequence b, and how many of them come from the cache.
 // Without APPEND: the first min(max(seqlens[b], 0), cap) cache rows.  With
@@ -169,45 +165,15 @@ __device__ __forceinline__ DecItem dec_item(const DecParams& p, int HG, int GPK,
   return I;
 }
 
-// Sums each of the GP partial dot products over the LPK lanes of a key group
-// and leaves every lane with all GP totals.  For GP = 4 and LPK = 8 the sums
-// are transposed while they are reduced (lane bits 2 and 1 pick which heads a
-// lane keeps), so that 4 shuffles + 4 adds give each lane one head's total and
-// 3 more shuffles collect the other three.
-template <int GP, int LPK>
-__device__ __forceinline__ void reduce_scores(float (&sc)[GP], int lane) {
-  if constexpr (GP == 4 && (LPK == 8 || LPK == 16)) {
-    // the two highest lane bits of the group (H = LPK/2, H/2) choose the kept head
-    constexpr int H = LPK / 2;
-    const bool bh = lane & H, bl = lane & (H / 2);
-    float k0 = bh ? sc[2] : sc[0], k1 = bh ? sc[3] : sc[1];
-    const float s0 = bh ? sc[0] : sc[2], s1 = bh ? sc[1] : sc[3];
-    k0 += __shfl_xor_sync(0xffffffffu, s0, H);
-    k1 += __shfl_xor_sync(0xffffffffu, s1, H);
-    float kept = bl ? k1 : k0;
-    kept += __shfl_xor_sync(0xffffffffu, bl ? k0 : k1, H / 2);
-#pragma unroll
-    for (int o = H / 4; o >= 1; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
-    // lane holds head (bh, bl) summed over the group; collect all four
-    const int base = lane & ~(LPK - 1);
-#pragma unroll
-    for (int g = 0; g < 4; ++g) sc[g] = __shfl_sync(0xffffffffu, kept, base + g * (H / 2));
-  } else {
-#pragma unroll
-    for (int o = 1; o < LPK; o <<= 1)
-#pragma unroll
-      for (int g = 0; g < GP; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], o);
-  }
-}
-
 template <int D, int GP, bool PAGED, bool APPEND>
 __global__ void __launch_bounds__(DecCfg<D, GP>::THREADS, DecCfg<D, GP>::CTAS_PER_SM)
 decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const DecParams p) {
   using C = DecCfg<D, GP>;
-  constexpr int NS = C::NS, T = C::T, LPK = C::LPK, KPW = C::KPW, NW = C::NW;
+  constexpr int NS = C::NS, T = C::T, NW = C::NW;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  // the 128-byte swizzle repeats every 1024 bytes: tiles start on such a boundary
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* mrg = reinterpret_cast<float*>(smem + NS * C::STAGE_BYTES);
   volatile int* item_w = reinterpret_cast<volatile int*>(smem + C::ITEM_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -294,9 +260,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (!((use >> s) & 1u)) continue;
-            tma_load_4d(dst + s * p.sub_rows * D * 2, &tm_k, &full[slot], 0, I.hkv, rows[s], pages[s]);
-            tma_load_4d(dst + C::TILE_BYTES + s * p.sub_rows * D * 2, &tm_v, &full[slot], 0, I.hkv, rows[s],
-                        pages[s]);
+#pragma unroll
+            for (int db = 0; db < D / 64; ++db) {   // 64 dimensions (128 bytes) per box
+              const int off = db * C::BLOCK_BYTES + s * p.sub_rows * 128;
+              tma_load_4d(dst + off, &tm_k, &full[slot], db * 64, I.hkv, rows[s], pages[s]);
+              tma_load_4d(dst + C::TILE_BYTES + off, &tm_v, &full[slot], db * 64, I.hkv, rows[s], pages[s]);
+            }
           }
         }
         ++it;
@@ -309,9 +278,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
 
   // -------------------------------------------------------------- consumers --
-  const int kg = lane / LPK;                    // key slot within a warp step
-  const int ds = lane % LPK;                    // 16-byte chunk: dimensions 8*ds .. 8*ds+7
-  constexpr int KS = (T / NW) / KPW;            // keys per lane group per tile
+  // Fragment coordinates (mma.sync m16n8): row g = query head of the group
+  // (rows >= GP are padding), columns 2 t4, 2 t4 + 1 = keys (scores) or
+  // dimensions (output).
+  const int g = lane >> 2, t4 = lane & 3;
+  constexpr int KSTEPS = D / 16, NT = D / 8;
+  const bool row_real = g < GP;
+  const uint32_t ring_base = smem_u32(smem);
   DecCursor cur{0, 0};
   int it = 0;                                   // ring slots consumed so far
   int ni = 0;                                   // items taken from the queue
@@ -331,173 +304,175 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const DecItem I = dec_item<T, APPEND>(p, HG, GPK, b, u);
     const int hq0 = I.hkv * G + (I.hg % GPK) * GP;
 
-    float qf[GP][8];
+    // Q of head g as the A fragment: per 16-dimension step, dims 2 t4.. and 2 t4 + 8..
+    uint32_t qa[KSTEPS][2];
+    {
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          p.q + (static_cast<size_t>(b) * p.Hq + hq0 + (row_real ? g : 0)) * D);
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + hq0 + g) * D);
-      bf16x8_to_f32(qrow[ds], qf[g]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        qa[ks][0] = row_real ? qrow[ks * 8 + t4] : 0u;
+        qa[ks][1] = row_real ? qrow[ks * 8 + 4 + t4] : 0u;
+      }
     }
-    float m[GP], l[GP], acc[GP][8];
+    float m_run = -INFINITY, l = 0.f, lr = 0.f;   // l, lr: this lane's share of the row sums
+    float o[NT][4];
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      m[g] = -INFINITY; l[g] = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-    }
+    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
-    // Per tile, a lane group owns KS keys (kt = warp*T/NW + st*KPW + kg).  Their
-    // scores are formed first (independent, so their reductions overlap), then
-    // one tile max per head decides a (rare) rescale, then p and the P.V update.
     for (int i = 0; ok && i < I.ntiles; ++i) {
       const int s = it % NS;
       if (!(ok = mbar_wait_warp(&full[s], (it / NS) & 1, lim, W_DEC_FULL))) break;
-      const uint8_t* ks = smem + s * C::STAGE_BYTES;
-      const uint8_t* vs = ks + C::TILE_BYTES;
+      const uint32_t kt = ring_base + s * C::STAGE_BYTES;
+      const uint32_t vt = kt + C::TILE_BYTES;
       const int key0 = I.k_begin + i * T;
-      const bool full_tile = key0 + T <= I.c_end;
-      float sc[KS][GP];
+      // V rows of this warp's keys at or past the item's last cache row hold
+      // stale or never-written data; their p is 0, but 0 * NaN is not, so they
+      // are cleared before the products read them
+      const bool partial = key0 + warp * 8 + 8 > I.c_end;
+      if (partial) {
+        const int kr = warp * 8 + (lane >> 2);      // 4 lanes per row, 32 bytes each per block
+        if (key0 + (kr - warp * 8) + warp * 8 >= I.c_end) {
 #pragma unroll
-      for (int st = 0; st < KS; ++st) {
-        const int kt = warp * (T / NW) + st * KPW + kg;
-        float kf[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(ks + kt * D * 2 + ds * 16), kf);
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1], a0, a1);
-          sc[st][g] = a0 + a1;
-        }
-      }
-#pragma unroll
-      for (int st = 0; st < KS; ++st) reduce_scores<GP, LPK>(sc[st], lane);
-      if (!full_tile) {                           // rows past the item's cache rows do not count
-#pragma unroll
-        for (int st = 0; st < KS; ++st) {
-          const int kt = warp * (T / NW) + st * KPW + kg;
-          if (key0 + kt >= I.c_end) {
-#pragma unroll
-            for (int g = 0; g < GP; ++g) sc[st][g] = -INFINITY;
+          for (int db = 0; db < D / 64; ++db) {
+            uint4* row = reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES + C::TILE_BYTES + db * C::BLOCK_BYTES + kr * 128);
+            row[(lane & 3) * 2] = make_uint4(0u, 0u, 0u, 0u);
+            row[(lane & 3) * 2 + 1] = make_uint4(0u, 0u, 0u, 0u);
           }
         }
+        __syncwarp();
       }
+      // S = Q K^T for this warp's keys 8 warp .. 8 warp + 7, two 16-dimension steps per ldmatrix
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int kr = warp * 8 + (lane & 7);       // key row this lane addresses
+        const int mi = lane >> 3;                   // which of the four 8x8 matrices
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float mt = sc[0][g];
-#pragma unroll
-        for (int st = 1; st < KS; ++st) mt = fmaxf(mt, sc[st][g]);
-        if (mt > m[g] + DEC_TAU) {                // false while both are -inf
-          const float a = ex2_approx(m[g] - mt);
-          l[g] *= a;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[g][e] *= a;
-          m[g] = mt;
+        for (int ks = 0; ks < KSTEPS; ks += 2) {
+          const int ksm = ks + (mi >> 1);
+          const int cc = (ksm & 3) * 2 + (mi & 1);  // 16-byte chunk (8 dimensions) in the 128-byte row
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kt + (ksm >> 2) * C::BLOCK_BYTES + kr * 128 + ((cc ^ (kr & 7)) << 4), b0, b1, b2, b3);
+          mma_16816(sc, qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+          mma_16816(sc, qa[ks + 1][0], 0u, qa[ks + 1][1], 0u, b2, b3);
         }
       }
+      const int kc = key0 + warp * 8 + 2 * t4;      // keys of this lane's two scores
+      float s0 = (kc < I.c_end) ? sc[0] * p.scale_log2 : -INFINITY;
+      float s1 = (kc + 1 < I.c_end) ? sc[1] * p.scale_log2 : -INFINITY;
+      float mt = fmaxf(s0, s1);
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const bool resc = mt > m_run + DEC_TAU;       // false while both are -inf
+      if (__any_sync(0xffffffffu, resc)) {
+        const float a = resc ? ex2_approx(m_run - mt) : 1.f;
+        l *= a; lr *= a;
 #pragma unroll
-      for (int st = 0; st < KS; ++st) {
-        const int kt = warp * (T / NW) + st * KPW + kg;
-        if (!full_tile && key0 + kt >= I.c_end) continue;   // never read V rows past the item's cache rows
-        float vf[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(vs + kt * D * 2 + ds * 16), vf);
+        for (int n = 0; n < NT; ++n) { o[n][0] *= a; o[n][1] *= a; }
+        if (resc) m_run = mt;
+      }
+      const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+      const float p0 = ex2_approx(s0 - msub), p1 = ex2_approx(s1 - msub);
+      const uint32_t pa = pack_bf16x2(p0, p1);
+      l += p0 + p1;
+      lr += __uint_as_float(pa << 16) + __uint_as_float(pa & 0xffff0000u);   // the rounded p, exactly
+      // O += P V: this warp's 8 keys x 8 dimensions per n-tile, four n-tiles per ldmatrix.trans
+      {
+        const int kr = warp * 8 + (lane & 7);
+        const int mi = lane >> 3;
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float pr = ex2_approx(sc[st][g] - m[g]);
-          l[g] += pr;
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1], acc[g][e], acc[g][e + 1]);
+        for (int n0 = 0; n0 < NT; n0 += 4) {
+          const int n = n0 + mi;                    // n-tile this lane addresses: dims 8n .. 8n + 7
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_trans(vt + (n >> 3) * C::BLOCK_BYTES + kr * 128 + (((n & 7) ^ (kr & 7)) << 4), v0, v1, v2, v3);
+          mma_1688(o[n0 + 0], pa, 0u, v0);
+          mma_1688(o[n0 + 1], pa, 0u, v1);
+          mma_1688(o[n0 + 2], pa, 0u, v2);
+          mma_1688(o[n0 + 3], pa, 0u, v3);
         }
       }
+      // generic writes to the slot (the cleared rows) come before the next TMA into it
+      if (partial) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       ++it;
     }
 
-    // the new token's key (APPEND): read from its input rows by warp 0, taken
-    // by key group 0 of that warp
+    // the new token's key (APPEND), in warp 0: scores from its input rows
     const bool has_new = APPEND && I.cached >= I.k_begin && I.cached < I.k_end;
     if (has_new && warp == 0 && ok) {
       const size_t nrow = (static_cast<size_t>(b) * p.Hkv + I.hkv) * D;
-      float kf[8], vf[8], sc[GP];
-      bf16x8_to_f32(reinterpret_cast<const uint4*>(p.k_new + nrow)[ds], kf);
-      bf16x8_to_f32(reinterpret_cast<const uint4*>(p.v_new + nrow)[ds], vf);
+      constexpr int DL = D / 32;                    // dimensions per lane in the dot products
+      float kf[DL];
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float a0 = 0.f, a1 = 0.f;
+      for (int e = 0; e < DL; ++e) kf[e] = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.k_new)[nrow + lane * DL + e]);
+      float snew = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) ffma2(a0, a1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1], a0, a1);
-        sc[g] = a0 + a1;
+      for (int h2 = 0; h2 < GP; ++h2) {
+        const __nv_bfloat16* qh = reinterpret_cast<const __nv_bfloat16*>(p.q) + (static_cast<size_t>(b) * p.Hq + hq0 + h2) * D;
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) d = fmaf(__bfloat162float(qh[lane * DL + e]), kf[e], d);
+#pragma unroll
+        for (int o2 = 16; o2 >= 1; o2 >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o2);
+        if (h2 == g) snew = d * p.scale_log2;
       }
-      reduce_scores<GP, LPK>(sc, lane);
-      if (kg == 0) {
+      // one more key for row g: the same online update as above
+      const bool rs = row_real && snew > m_run + DEC_TAU;
+      if (__any_sync(0xffffffffu, rs)) {
+        const float a = rs ? ex2_approx(m_run - snew) : 1.f;
+        l *= a; lr *= a;
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          if (sc[g] > m[g] + DEC_TAU) {
-            const float a = ex2_approx(m[g] - sc[g]);
-            l[g] *= a;
+        for (int n = 0; n < NT; ++n) { o[n][0] *= a; o[n][1] *= a; }
+        if (rs) m_run = snew;
+      }
+      const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+      const float pn = row_real ? ex2_approx(snew - msub) : 0.f;
+      const float pnr = __bfloat162float(__float2bfloat16_rn(pn));   // the rounded p, as in the products
+      if (t4 == 0) { l += pn; lr += pnr; }          // counted once per row (the quad's shares are summed)
+      const __nv_bfloat16* vn = reinterpret_cast<const __nv_bfloat16*>(p.v_new) + nrow;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] *= a;
-            m[g] = sc[g];
-          }
-          const float pr = ex2_approx(sc[g] - m[g]);
-          l[g] += pr;
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1], acc[g][e], acc[g][e + 1]);
-        }
+      for (int n = 0; n < NT; ++n) {
+        o[n][0] = fmaf(pnr, __bfloat162float(vn[n * 8 + 2 * t4]), o[n][0]);
+        o[n][1] = fmaf(pnr, __bfloat162float(vn[n * 8 + 2 * t4 + 1]), o[n][1]);
       }
     }
 
-    // merge the key groups of this warp (lanes ds, ds+LPK, ...)
-#pragma unroll
-    for (int o = LPK; o < 32; o <<= 1) {
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m[g], o);
-        const float lo = __shfl_xor_sync(0xffffffffu, l[g], o);
-        const float mn = fmaxf(m[g], mo);
-        const float a = (m[g] == -INFINITY) ? 0.f : ex2_approx(m[g] - mn);
-        const float c = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mn);
-        l[g] = l[g] * a + lo * c;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], o);
-          acc[g][e] = acc[g][e] * a + ao * c;
-        }
-        m[g] = mn;
-      }
-    }
+    // this warp's row sums: the four lanes of a row hold shares
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    lr += __shfl_xor_sync(0xffffffffu, lr, 1);
+    lr += __shfl_xor_sync(0xffffffffu, lr, 2);
     // the previous item's readers of the merge area are done
     asm volatile("bar.sync 1, %0;" :: "r"(NW * 32) : "memory");
-    // per-warp state to shared memory: [w][g] -> m, l, acc[D]
-    if (kg == 0) {
+    // per-warp state to shared memory: [w][g] -> m, l, lr, pad, O[D]
+    if (row_real) {
+      float* dst = mrg + (warp * GP + g) * C::MRG_STRIDE;
+      if (t4 == 0) { dst[0] = m_run; dst[1] = l; dst[2] = lr; }
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float* dst = mrg + (warp * GP + g) * (D + 2);
-        if (ds == 0) { dst[0] = m[g]; dst[1] = l[g]; }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) dst[2 + ds * 8 + e] = acc[g][e];
-      }
+      for (int n = 0; n < NT; ++n) { dst[4 + n * 8 + 2 * t4] = o[n][0]; dst[4 + n * 8 + 2 * t4 + 1] = o[n][1]; }
     }
     // every consumer warp leaves together if any of them gave up waiting
     if (!bar_sync_and(1, NW * 32, ok)) break;
     for (int idx = threadIdx.x; idx < GP * D; idx += NW * 32) {
-      const int g = idx / D, d = idx % D;
+      const int h2 = idx / D, d = idx % D;
       float mw[NW], mx = -INFINITY;
 #pragma unroll
-      for (int w2 = 0; w2 < NW; ++w2) { mw[w2] = mrg[(w2 * GP + g) * (D + 2)]; mx = fmaxf(mx, mw[w2]); }
-      float L = 0.f, O = 0.f;
+      for (int w2 = 0; w2 < NW; ++w2) { mw[w2] = mrg[(w2 * GP + h2) * C::MRG_STRIDE]; mx = fmaxf(mx, mw[w2]); }
+      float L = 0.f, LR = 0.f, O = 0.f;
 #pragma unroll
       for (int w2 = 0; w2 < NW; ++w2) {
-        const float* src = mrg + (w2 * GP + g) * (D + 2);
+        const float* src = mrg + (w2 * GP + h2) * C::MRG_STRIDE;
         const float a = (mw[w2] == -INFINITY) ? 0.f : ex2_approx(mw[w2] - mx);
         L = fmaf(src[1], a, L);
-        O = fmaf(src[2 + d], a, O);
+        LR = fmaf(src[2], a, LR);
+        O = fmaf(src[4 + d], a, O);
       }
-      const size_t prow = (static_cast<size_t>(b) * p.Hq + hq0 + g) * p.max_splits + I.split;
+      const size_t prow = (static_cast<size_t>(b) * p.Hq + hq0 + h2) * p.max_splits + I.split;
       if (!index_ok(prow, 1, static_cast<size_t>(p.B) * p.Hq * p.max_splits, W_IDX_DEC_PART)) continue;
-      p.o_part[prow * D + d] = L > 0.f ? O / L : 0.f;
+      // O is normalised by the sum of the rounded p that the products used, the
+      // LSE by the exact sum
+      p.o_part[prow * D + d] = LR > 0.f ? O / LR : 0.f;
       if (d == 0) p.lse_part[prow] = L > 0.f ? (mx + log2f(L)) * LN2 : -INFINITY;
     }
 
