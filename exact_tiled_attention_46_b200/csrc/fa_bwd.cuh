@@ -23,7 +23,8 @@
 //                   quadrant and take 64 of the 128 query columns each (no row
 //                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
 //                   on the tiles that need it; P^T is published first (the dV
-//                   products run while dS^T is formed from P read back)
+//                   products, then the next pair's S^T, run while dS^T is
+//                   formed from P kept in registers)
 //        warps 8-11 one thread per query row: dQ tile from TMEM (two buffers at
 //                   D = 64) into a swizzled shared-memory box per warp, added to
 //                   the fp32 accumulator by TMA reduce-add (32 rows x 32
@@ -53,7 +54,7 @@ struct BwdCfg {
   // dQ staging: per read-out warp two 4 KB boxes (32 rows x 32 fp32, 128-byte swizzle)
   static constexpr int DQS_OFF = ROW_OFF + NQ * 1024;
   static constexpr int BAR_OFF = DQS_OFF + 4 * 8192;
-  static constexpr int NBARS = 1 + 2 * NQ + 4 + 4 + 2;
+  static constexpr int NBARS = 1 + 2 * NQ + 5 + 4 + 2;
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
@@ -146,8 +147,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = q_full + NQ;
-  uint64_t* sdp_full = q_empty + NQ;
-  uint64_t* p_ready = sdp_full + 1;
+  uint64_t* s_full = q_empty + NQ;                // S^T of the pair is in TMEM
+  uint64_t* dp_full = s_full + 1;                 // dP^T of the pair is in TMEM
+  uint64_t* p_ready = dp_full + 1;
   uint64_t* ds_ready = p_ready + 1;
   uint64_t* ds_free = ds_ready + 1;
   uint64_t* dq_full = ds_free + 1;       // [2]
@@ -179,7 +181,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < NQ; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
-    mbar_init(sdp_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
     mbar_init(p_ready, 256);
     mbar_init(ds_ready, 256);
     mbar_init(ds_free, 1);
@@ -234,24 +237,30 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t k_base = smem_u32(smem + C::K_OFF), v_base = smem_u32(smem + C::V_OFF);
       const uint32_t q_base = smem_u32(smem + C::Q_OFF), ds_base = smem_u32(smem + C::DS_OFF);
       const uint32_t dslo_base = smem_u32(smem + C::DSLO_OFF);
-      // P^T part of queries 16kk..16kk+15 in TMEM: chunk (kk / 4, (kk % 4) / 2) of 32
-      // query columns holds P_hi in its first 16 columns and P_lo in the next 16
-      auto p_col = [](int kk) { return C::T_S + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8; };
+      // P^T of queries 16kk..16kk+15 in TMEM: P_hi in columns 16kk..16kk+7, P_lo
+      // in the next 8 (over the S^T columns of those queries)
+      auto p_col = [](int kk) { return C::T_S + kk * 16; };
       auto kmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
       auto mnmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + kk * 2048, 16384, 1024); };
-      auto issue_s_dp = [&](int n) {
-        const uint32_t qa = q_base + (n % NQ) * 2 * C::TILE, da = qa + C::TILE;
+      auto issue_s = [&](int n) {
+        const uint32_t qa = q_base + (n % NQ) * 2 * C::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_S, kmaj(k_base, kk), kmaj(qa, kk), ID_SS, kk > 0);
+        umma_commit(s_full);
+      };
+      auto issue_dp = [&](int n) {
+        const uint32_t da = q_base + (n % NQ) * 2 * C::TILE + C::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_DP, kmaj(v_base, kk), kmaj(da, kk), ID_SS, kk > 0);
+        umma_commit(dp_full);
       };
       bool ok = mbar_wait(kv_full, 0, lim, W_BWD_KV) && mbar_wait(&q_full[0], 0, lim, W_BWD_QF);
       tc_fence_after();
-      if (ok) { issue_s_dp(0); umma_commit(sdp_full); }
+      if (ok) { issue_s(0); issue_dp(0); }
       for (int n = 0; ok && n < npairs; ++n) {
         const int s = n % NQ, bq = n % NB;
         const uint32_t qa = q_base + s * 2 * C::TILE, da = qa + C::TILE;
+        const bool more = n + 1 < npairs;
         if (!(ok = mbar_wait(p_ready, n & 1, lim, W_BWD_P))) break;
         tc_fence_after();
 #pragma unroll
@@ -259,16 +268,19 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           umma_ts(tmem + C::T_DV, tmem + p_col(kk), mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dV += P_lo^T dO
-          umma_ts(tmem + C::T_DV, tmem + p_col(kk) + 16, mnmaj(da, kk), ID_DVK, 1u);
-        if (!(ok = mbar_wait(ds_ready, n & 1, lim, W_BWD_DS))) break;
-        tc_fence_after();
-        const bool more = n + 1 < npairs;
-        if (!C::DQ_IN_DP && more) {         // next pair's S^T, dP^T first: the compute warps start early
+          umma_ts(tmem + C::T_DV, tmem + p_col(kk) + 8, mnmaj(da, kk), ID_DVK, 1u);
+        // the next pair's S^T goes over P^T as soon as the dV products are issued
+        // (the pipe runs them in order; the compute warps keep P in registers),
+        // when its Q has a stage of its own (with one stage, Q(n+1) replaces
+        // Q(n) only after this pair's last product)
+        if (more && NQ > 1) {
           if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
           tc_fence_after();
-          issue_s_dp(n + 1);
-          umma_commit(sdp_full);
+          issue_s(n + 1);
         }
+        if (!(ok = mbar_wait(ds_ready, n & 1, lim, W_BWD_DS))) break;
+        tc_fence_after();
+        if (!C::DQ_IN_DP && more) issue_dp(n + 1);   // dP^T was read by the dS^T phase
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dK += dS_hi^T Q  (K = 128 queries)
           umma_ss(tmem + C::T_DK, kmaj(ds_base, kk), mnmaj(qa, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
@@ -287,11 +299,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         umma_commit(&q_empty[s]);
         if (C::DQ_IN_DP && more) {          // dP^T(n+1) overwrites dQ(n): wait for its read-out
           if (!(ok = mbar_wait(&dq_free[0], n & 1, lim, W_BWD_DQF))) break;
+          tc_fence_after();
+        }
+        if (more && NQ == 1) {
           if (!(ok = mbar_wait(&q_full[(n + 1) % NQ], ((n + 1) / NQ) & 1, lim, W_BWD_QF))) break;
           tc_fence_after();
-          issue_s_dp(n + 1);
-          umma_commit(sdp_full);
+          issue_s(n + 1);
         }
+        if (C::DQ_IN_DP && more) issue_dp(n + 1);
       }
       umma_commit(dkv_done);
       umma_commit(mma_done);
@@ -314,26 +329,28 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int i = i0 + n / G;
       const float* lse2 = reinterpret_cast<const float*>(smem + C::ROW_OFF + s * 1024);
       const float* dlt = lse2 + 128;
-      if (!mbar_wait_warp(sdp_full, n & 1, lim, W_BWD_SDP)) break;
+      if (!mbar_wait_warp(s_full, n & 1, lim, W_BWD_SDP)) break;
       tc_fence_after();
       // allowed when key <= query + off, i.e. column c >= cmin (nothing for keys past Lk)
       const int cmin = key < p.Lk ? (CAUSAL ? key - off - i * 128 : -1) : (1 << 30);
       const int rowoff = r * 128;
       bool ok = true;
-      // Phase 1: P^T = 2^(S^T * scale - LSE) (masked), as P_hi + P_lo over the
-      // S^T columns it comes from; published at once, so that the dV products
-      // run while phase 2 forms dS^T.
+      // Phase 1: P^T = 2^(S^T * scale - LSE) (masked) for this warp's 64 query
+      // columns, 16 at a time: kept in registers (fp32) for phase 2 and stored
+      // as P_hi + P_lo over the 16 S^T columns they come from, the A operand of
+      // the dV products; published at once.
+      float pv[64];
 #pragma unroll
-      for (int lc = 0; lc < 2; ++lc) {
-        const int c0 = hh * 64 + lc * 32;              // first query column of this chunk
-        uint32_t sv[32];
-        tmem_ld_32x32b_x32(tmem + lane_bits + C::T_S + c0, sv);
+      for (int sc = 0; sc < 4; ++sc) {
+        const int c0 = hh * 64 + sc * 16;              // first query column of this sub-chunk
+        uint32_t sv[16];
+        tmem_ld_32x32b_x16(tmem + lane_bits + C::T_S + c0, sv);
         // the mask only matters where some key row of the warp starts after c0
         // (the causal diagonal, keys past Lk); elsewhere every column is allowed
         const bool masked = __any_sync(0xffffffffu, cmin > c0);
-        uint32_t phi[16], plo[16];
+        uint32_t phi[8], plo[8];
 #pragma unroll
-        for (int t4 = 0; t4 < 8; ++t4) {
+        for (int t4 = 0; t4 < 4; ++t4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + 4 * t4);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
@@ -347,64 +364,59 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               p0 = (c >= cmin) ? p0 : 0.f;
               p1 = (c + 1 >= cmin) ? p1 : 0.f;
             }
+            pv[sc * 16 + 2 * t] = p0;
+            pv[sc * 16 + 2 * t + 1] = p1;
             phi[t] = pack_bf16x2(p0, p1);
             float r0, r1;
             resid_bf16x2(phi[t], p0, p1, r0, r1);
             plo[t] = pack_bf16x2(r0, r1);
           }
         }
-        // P_hi and P_lo of query columns [c0, c0+32) go back over the 32 S^T columns
-        // just read: P_hi to the first 16, P_lo to the next 16
-        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + c0, phi);
-        tmem_st_32x32b_x16(tmem + lane_bits + C::T_S + c0 + 16, plo);
+        tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + c0, phi);
+        tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + c0 + 8, plo);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready);
-      // Phase 2: dS^T = P^T * (dP^T - Delta), P^T = P_hi + P_lo read back, as
-      // dS_hi + dS_lo into swizzled shared memory.
+      // Phase 2: dS^T = P^T * (dP^T - Delta) into swizzled shared memory as
+      // dS_hi + dS_lo, 16 query columns at a time.
+      if (!mbar_wait_warp(dp_full, n & 1, lim, W_BWD_SDP)) break;
+      tc_fence_after();
 #pragma unroll
-      for (int lc = 0; lc < 2; ++lc) {
-        const int c0 = hh * 64 + lc * 32;
-        uint32_t dp[32], ph[16], pl[16];
-        tmem_ld_32x32b_x32_nowait(tmem + lane_bits + C::T_DP + c0, dp);
-        tmem_ld_32x32b_x16_nowait(tmem + lane_bits + C::T_S + c0, ph);
-        tmem_ld_32x32b_x16_nowait(tmem + lane_bits + C::T_S + c0 + 16, pl);
-        tmem_ld_wait_regs(dp);
-        tmem_ld_wait_regs(ph);
-        tmem_ld_wait_regs(pl);
-        uint32_t dhi[16], dlo[16];
+      for (int sc = 0; sc < 4; ++sc) {
+        const int c0 = hh * 64 + sc * 16;
+        uint32_t dp[16];
+        tmem_ld_32x32b_x16(tmem + lane_bits + C::T_DP + c0, dp);
+        uint32_t dhi[8], dlo[8];
 #pragma unroll
-        for (int t4 = 0; t4 < 8; ++t4) {
+        for (int t4 = 0; t4 < 4; ++t4) {
           const float4 d4 = *reinterpret_cast<const float4*>(dlt + c0 + 4 * t4);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = 2 * t4 + u;
-            float p0 = __uint_as_float(pl[t] << 16), p1 = __uint_as_float(pl[t] & 0xffff0000u);
-            add_bf16x2_f32(p0, p1, ph[t]);
             float e0, e1, s0, s1, r0, r1;
             fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -(u ? d4.z : d4.x),
                   -(u ? d4.w : d4.y));
-            ffma2(s0, s1, p0, p1, e0, e1, 0.f, 0.f);
+            ffma2(s0, s1, pv[sc * 16 + 2 * t], pv[sc * 16 + 2 * t + 1], e0, e1, 0.f, 0.f);
             dhi[t] = pack_bf16x2(s0, s1);
             resid_bf16x2(dhi[t], s0, s1, r0, r1);
             dlo[t] = pack_bf16x2(r0, r1);
           }
         }
         // the shared-memory operands of pair n - 1 must have been consumed
-        if (lc == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
-        // columns c0..c0+31: 4 16-byte chunks of the 128-byte row of block hh (128B swizzle)
+        if (sc == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
+        // query columns c0..c0+15: two 16-byte chunks of the 128-byte row of block hh (128B swizzle)
         const int blk = hh * 16384 + rowoff;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int o16 = blk + (((lc * 4 + t) ^ (r & 7)) << 4);
+        for (int t = 0; t < 2; ++t) {
+          const int o16 = blk + (((sc * 2 + t) ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(smem + C::DS_OFF + o16) = make_uint4(dhi[4 * t], dhi[4 * t + 1], dhi[4 * t + 2], dhi[4 * t + 3]);
           *reinterpret_cast<uint4*>(smem + C::DSLO_OFF + o16) = make_uint4(dlo[4 * t], dlo[4 * t + 1], dlo[4 * t + 2], dlo[4 * t + 3]);
         }
       }
       if (!ok) break;
       fence_proxy_async_smem();
-      tc_fence_before();                               // the phase-2 reads of P and dP^T come first
+      tc_fence_before();                               // the phase-2 reads of dP^T come first
       mbar_arrive(ds_ready);
     }
     setmaxnreg_dec<BWD_LAUNCH_REGS>();
