@@ -52,24 +52,24 @@ NOMINAL_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0,
 # its units of work (see the profiles/ summaries for the captured case).
 PROFILED_TRAFFIC = {
     "fwd_kernel causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
-                                  "sha256_16": "88f18afadce39b9c", "bytes": 127665408 + 9809152},
+                                  "sha256_16": "644cd20e74d80560", "bytes": 126125824 + 9488384},
     "fwd_kernel long_gqa_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
-                                    "sha256_16": "88f18afadce39b9c", "bytes": 340705024 + 98593280},
-    "bwd_main_kernel train_fwd_bwd": {"sources": ("csrc/fa_bwd.cuh", "csrc/sm100.cuh"),
-                                      "sha256_16": "3625827544788fa1", "bytes": 406916864 + 225205760},
+                                    "sha256_16": "644cd20e74d80560", "bytes": 352846080 + 97611776},
     "fwd_kernel<fp8> causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
-                                       "sha256_16": "ff576a2b73270a40", "bytes": 50417920 + 2505984},
+                                       "sha256_16": "644cd20e74d80560", "bytes": 50400256 + 3337728},
+    "bwd_main_kernel train_fwd_bwd": {"sources": ("csrc/fa_bwd.cuh", "csrc/sm100.cuh"),
+                                      "sha256_16": "c3e4fad1efd2fb24", "bytes": 407020032 + 225529344},
     # captured on the first 16 sequences of the decode workload (1.35888 GB of KV
     # rows), scaled to a launch by the KV bytes it reads
     "decode_split_kernel splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
-                                           "sha256_16": "475ed25160e6b429",
-                                           "bytes_per_kv_byte": (1360300288 + 8381952) / 1358876672},
+                                           "sha256_16": "cc6efd0dad8ce196",
+                                           "bytes_per_kv_byte": (1362351360 + 12924672) / 1358876672},
     "decode_split_kernel<append> splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
-                                                   "sha256_16": "475ed25160e6b429",
-                                                   "bytes_per_kv_byte": (1360314624 + 9055488) / 1358876672},
+                                                   "sha256_16": "cc6efd0dad8ce196",
+                                                   "bytes_per_kv_byte": (1366708480 + 19545344) / 1358876672},
     "decode_split_kernel<paged16> splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
-                                                    "sha256_16": "475ed25160e6b429",
-                                                    "bytes_per_kv_byte": (1359829248 + 8537088) / 1358876672},
+                                                    "sha256_16": "cc6efd0dad8ce196",
+                                                    "bytes_per_kv_byte": (1362181376 + 13036544) / 1358876672},
 }
 
 
