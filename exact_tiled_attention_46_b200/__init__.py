@@ -337,7 +337,7 @@ def selftest_wait_timeout(wait_ns: int, device=None):
 
 
 def launch_guard(bwd: bool, D: int, causal: bool, query_regs: bool = True):
-    """(compiled registers or None, registers the split assumes, cached verdict) of one kernel instantiation."""
+    """(compiled registers or None, registers the split assumes, cached check result) of one kernel instantiation."""
     regs, exp, state = ctypes.c_int(-1), ctypes.c_int(0), ctypes.c_int(0)
     _check(lib().fa_launch_guard(int(bool(bwd)), int(D), int(bool(causal)),
                                  ctypes.byref(regs) if query_regs else None, ctypes.byref(exp), ctypes.byref(state)),

@@ -126,7 +126,7 @@ __global__ void selftest_exp2_poly_kernel(const float* x, float* y, int n) {
 // The forward and backward kernels move registers between warpgroups
 // (setmaxnreg); that is only safe when the launch allocation per thread is
 // exactly the one the split was computed for.  A build that allocates
-// differently is refused, never run.  The verdict is kept per kernel
+// differently is refused, never run.  The result is kept per kernel
 // instantiation (each launch_* template instance owns its `state`), because
 // all instantiations of one kernel template share a function type.
 enum : int { REGS_UNKNOWN = 0, REGS_MATCH = 1, REGS_MISMATCH = 2 };

@@ -285,7 +285,7 @@ fa_status fa_selftest_wait_timeout(unsigned long long wait_ns, fa_stream_t strea
  * compares the compiled register count with that figure and refuses the launch
  * (FA_ERR_UNSUPPORTED) on a mismatch.  For the instantiation (bwd, D, causal)
  * this reports, when the pointers are not NULL: *state, that instantiation's
- * cached verdict (0 not yet checked, 1 match, 2 mismatch; never changed by
+ * cached check result (0 not yet checked, 1 match, 2 mismatch; never changed by
  * this call); *expected_regs, the figure the split assumes; *num_regs, the
  * compiled count (queried from the runtime, which needs a GPU; pass NULL to
  * skip).  D must be 64 or 128, or -128 for the e4m3 forward (bwd = 0).  No

@@ -144,7 +144,7 @@ def test_exp2_selftest_rejects_bad_arguments(L):
 
 
 def test_launch_guard_reports_per_instantiation_state_without_gpu(L):
-    """Before any launch every kernel instantiation's register verdict is
+    """Before any launch every kernel instantiation's register check result is
     'not yet checked'; querying it (without the compiled count, which needs a
     GPU) changes nothing."""
     for bwd in (0, 1):

@@ -4,7 +4,7 @@ The forward and backward kernels move registers between warpgroups with
 setmaxnreg, which is only safe when each thread is launched with exactly the
 registers the split assumes.  Every instantiation (forward / backward, D 64 /
 128, causal or not) must compile to that count, and the library must check
-each instantiation itself before its first launch rather than let one verdict
+each instantiation itself before its first launch rather than let one result
 stand for all kernels of the same function type.
 """
 import os

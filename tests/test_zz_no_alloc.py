@@ -16,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import exact_tiled_attention_46_b200 as fa
 from exact_tiled_attention_46_b200 import inputs as synth
 
@@ -58,6 +59,11 @@ def test_no_alloc_decode_matches_regular_on_two_calls():
         torch.cuda.synchronize()
         check_close(f64(out), f64(ref_o), bf16_output=False, what="no-alloc O")
         check_lse(f64(lse), f64(ref_l), what="no-alloc LSE")
+        # and against the CPU fp64 oracle directly
+        ro, rl = oracle.attn_decode(synth.as_f64(x["q"]), synth.as_f64(x["k_cache"]), synth.as_f64(x["v_cache"]),
+                                    x["seqlens"].numpy(), scale)
+        check_close(f64(out), ro, bf16_output=False, what="no-alloc O vs oracle")
+        check_lse(f64(lse), rl, what="no-alloc LSE vs oracle")
 
 
 def test_no_alloc_decode_rejects_configurations_beyond_the_scratch():
