@@ -58,7 +58,7 @@ PROFILED_TRAFFIC = {
     "fwd_kernel<fp8> causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
                                        "sha256_16": "644cd20e74d80560", "bytes": 50400256 + 3337728},
     "bwd_main_kernel train_fwd_bwd": {"sources": ("csrc/fa_bwd.cuh", "csrc/sm100.cuh"),
-                                      "sha256_16": "c3e4fad1efd2fb24", "bytes": 407020032 + 225529344},
+                                      "sha256_16": "0a8b5887803d96cb", "bytes": 406922240 + 224315904},
     # captured on the first 16 sequences of the decode workload (1.35888 GB of KV
     # rows), scaled to a launch by the KV bytes it reads
     "decode_split_kernel splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),
@@ -305,7 +305,9 @@ def section_train(fa, steps, warmup, flush, stream, peaks, peak_src, dev):
             "roofline": roofline("tensor", tfb, peaks, peak_src, "TFLOP/s",
                                  traffic=profiled_traffic("bwd_main_kernel train_fwd_bwd"),
                                  algorithmic_bytes=bwd_bytes),
-            "roofline_note": "backward call (pre-pass, main kernel, dQ post-pass); traffic is the main kernel's"}
+            "roofline_note": "backward call (input maxima, pre-pass, main kernel, dQ post-pass); traffic is the "
+                             "main kernel's; its products run on fp16 (same tensor rate as bf16)",
+            "dtype": "bf16 in and out; fp16 products (power-of-two scaled inputs), fp32 accumulate"}
 
 
 def section_decode(fa, steps, warmup, flush, stream, peaks, peak_src, dev):

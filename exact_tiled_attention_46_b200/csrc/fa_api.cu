@@ -486,8 +486,10 @@ fa_status fa_decode_splitkv_static(const void* q, const void* k_cache, const voi
 size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D) {
   if (B <= 0 || Hq <= 0 || Lq < 0 || D <= 0) return 0;
   const size_t lq_pad = align_up(size_t(Lq), 128);
-  // fp32 dQ accumulator, then the padded log2 LSE and Delta rows
-  return align_up(size_t(B) * Lq * Hq * D * 4, 256) + 2 * align_up(size_t(B) * Hq * lq_pad * 4, 256);
+  // fp32 dQ accumulator, the padded log2 LSE and Delta rows, the scaled fp16
+  // copies of q and dO, the four input maxima
+  return align_up(size_t(B) * Lq * Hq * D * 4, 256) + 2 * align_up(size_t(B) * Hq * lq_pad * 4, 256) +
+         2 * align_up(size_t(B) * Lq * Hq * D * 2, 256) + 256;
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -518,25 +520,42 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   const int lq_pad = static_cast<int>(align_up(size_t(Lq), 128));
   const size_t acc_bytes = size_t(B) * Lq * Hq * D * 4;
   const size_t row_bytes = align_up(size_t(B) * Hq * lq_pad * 4, 256);
-  float* dq_acc = static_cast<float*>(workspace);
-  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + align_up(acc_bytes, 256));
+  const size_t h_bytes = align_up(size_t(B) * Lq * Hq * D * 2, 256);
+  char* ws = static_cast<char*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + align_up(acc_bytes, 256));
   float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + row_bytes);
-  if (cudaMemsetAsync(dq_acc, 0, acc_bytes, st) != cudaSuccess) return FA_ERR_CUDA;
+  uint16_t* q16 = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(delta) + row_bytes);
+  uint16_t* do16 = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(q16) + h_bytes);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(do16) + h_bytes);
+  if (cudaMemsetAsync(dq_acc, 0, acc_bytes, st) != cudaSuccess || cudaMemsetAsync(amax, 0, 16, st) != cudaSuccess)
+    return FA_ERR_CUDA;
   {
-    const size_t rows = size_t(B) * lq_pad * Hq;
-    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 255) / 256, 148 * 16));
+    const size_t nq = size_t(B) * Lq * Hq * D, nk = size_t(B) * Lk * Hkv * D;
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((std::max(nq, nk) / 8 + 1023) / 1024, 148 * 4));
+    fa::bwd_amax_kernel<<<dim3(blocks, 4), 256, 0, st>>>(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                                static_cast<const uint16_t*>(v), static_cast<const uint16_t*>(dO),
+                                                nq, nk, amax);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  {
+    const size_t chunks = size_t(B) * lq_pad * Hq * (D / 8);         // one thread per 16-byte chunk of a row
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((chunks + 255) / 256, 148 * 16));
     fa::bwd_pre_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dO),
-                                               lse, lse2, delta, B, Hq, Lq, lq_pad, D);
+                                               static_cast<const uint16_t*>(q), lse, amax, lse2, delta, q16, do16, B,
+                                               Hq, Lq, lq_pad, D);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   CUtensorMap mq, mk, mv, mdo, mdq;
-  // the fp32 dQ accumulator takes reductions of 32-row x 32-column boxes
-  if (!map_bshd(&mq, q, B, Lq, Hq, D, 64, 128, true) || !map_bshd(&mk, k, B, Lk, Hkv, D, 64, 128, true) ||
-      !map_bshd(&mv, v, B, Lk, Hkv, D, 64, 128, true) || !map_bshd(&mdo, dO, B, Lq, Hq, D, 64, 128, true) ||
+  // q and dO are read from their fp16 copies (2-byte elements: the bf16 map
+  // type only sets the element size here), k and v as given; the fp32 dQ
+  // accumulator takes reductions of 32-row x 32-column boxes
+  if (!map_bshd(&mq, q16, B, Lq, Hq, D, 64, 128, true) || !map_bshd(&mk, k, B, Lk, Hkv, D, 64, 128, true) ||
+      !map_bshd(&mv, v, B, Lk, Hkv, D, 64, 128, true) || !map_bshd(&mdo, do16, B, Lq, Hq, D, 64, 128, true) ||
       !map_bshd(&mdq, dq_acc, B, Lq, Hq, D, 32, 32, true, true))
     return FA_ERR_CUDA;
   fa::BwdParams p;
-  p.lse2 = lse2; p.delta = delta; p.dk = dk; p.dv = dv;
+  p.lse2 = lse2; p.delta = delta; p.amax = amax; p.dk = dk; p.dv = dv;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.Lq_pad = lq_pad;
   p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f; p.g_fp32 = (grad_dtype == FA_FP32);
   p.wait_limit_ns = g_wait_limit_ns.load();
@@ -547,7 +566,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (s != FA_OK) return s;
   const size_t n = size_t(B) * Lq * Hq * D;
   const unsigned blocks = static_cast<unsigned>(std::min<size_t>((n / 4 + 255) / 256, 148 * 16));
-  fa::bwd_post_kernel<<<blocks, 256, 0, st>>>(dq_acc, dq, n, scale, grad_dtype == FA_FP32);
+  fa::bwd_post_kernel<<<blocks, 256, 0, st>>>(dq_acc, dq, n, scale, amax, D, grad_dtype == FA_FP32);
   return launch_status();
 }
 

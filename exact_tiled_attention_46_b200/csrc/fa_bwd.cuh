@@ -6,19 +6,28 @@
 //     dV = P^T dO,   dP = dO V^T,   Delta_i = sum_d dO_id O_id,
 //     dS = P * (dP - Delta),   dQ = scale dS K,   dK = scale dS^T Q.
 //
-// Three launches on the caller's stream (plus a memset of the dQ accumulator):
+// The products run on fp16 operands.  Every bf16 input value is an fp16 value
+// once scaled by a power of two into fp16's range, so each input tensor is
+// scaled by 2^k (from its largest magnitude) and converted exactly: Q, K, V to
+// a largest magnitude in [2^7, 2^8), dO so that |dP|, |Delta| and |dS| stay
+// below 2^15.  P^T and dS^T enter the products as single fp16 values (10
+// fraction bits); the scales come out exactly at the end.
+//
+// Four launches on the caller's stream (plus memsets of the dQ accumulator and
+// of the four maxima):
+//   bwd_amax_kernel  the largest |q|, |k|, |v|, |dO|.
 //   bwd_pre_kernel   Delta, the LSE in log2 units (+inf for rows without a key,
-//                    so that their P is 0), both padded to 128-row tiles.
+//                    so that their P is 0), both padded to 128-row tiles; the
+//                    scaled fp16 copies of q and dO.
 //   bwd_main_kernel  one CTA per (batch, kv head, 128-key tile), head-major; loops over the
 //                    (query tile, query head of the group) pairs:
-//        warp 12    TMA: K, V once; Q, dO, LSE, Delta per pair (NQ stages)
+//        warp 12    TMA: K, V once (bf16, converted to scaled fp16 in place by
+//                   warps 0-7); Q, dO (fp16 copies), LSE, Delta per pair
+//                   (NQ stages)
 //        warp 13    tcgen05: S^T = K Q^T and dP^T = V dO^T into TMEM,
 //                   dV += P^T dO, dK += dS^T Q, dQ = dS K
-//        P^T and dS^T enter the products as bf16.  P^T = P_hi + P_lo and
-//        dS^T = dS_hi + dS_lo (each part bf16; P_hi and P_lo in TMEM over the
-//        S^T columns they come from, dS_hi and dS_lo in swizzled shared
-//        memory); dV and dK take both parts, so that their only rounding is the
-//        fp32 accumulation, and dQ takes dS_hi.
+//        P^T (fp16) goes to TMEM over the S^T columns it comes from, dS^T
+//        (fp16) to swizzled shared memory.
 //        warps 0-7  one thread per key row; warps w and w + 4 share a TMEM lane
 //                   quadrant and take 64 of the 128 query columns each (no row
 //                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
@@ -31,12 +40,26 @@
 //                   columns per operation); at the end dK, dV out of TMEM
 //        warp 14    TMEM allocation; warp 15 idles.  The control warpgroup
 //                   (12-15) lends registers to the other three.
-//   bwd_post_kernel  dQ = scale * accumulator, converted to the output dtype.
+//   bwd_post_kernel  dQ = scale * accumulator (with the input scales taken
+//                    out), converted to the output dtype.
 #pragma once
 #include "sm100.cuh"
 #include "fa.h"
 
 namespace fa {
+
+// Instruction descriptor, kind::f16 with A and B fp16 (format 0), D fp32;
+// bits as for idesc_bf16_f32.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) |
+         (uint32_t(M >> 4) << 24);
+}
+// Two floats rounded (nearest even) to fp16, packed with lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 
 template <int D>
 struct BwdCfg {
@@ -48,13 +71,13 @@ struct BwdCfg {
   static constexpr int V_OFF = TILE;
   static constexpr int Q_OFF = 2 * TILE;              // stage s: Q at +s*2*TILE, dO after it
   static constexpr int DS_OFF = Q_OFF + NQ * 2 * TILE;
-  static constexpr int DS_BYTES = 128 * 128 * 2;     // one 128 x 128 bf16 operand (128B swizzle)
-  static constexpr int DSLO_OFF = DS_OFF + DS_BYTES;  // low bf16 part of dS^T
-  static constexpr int ROW_OFF = DSLO_OFF + DS_BYTES; // stage s: lse2[128], delta[128]
+  static constexpr int DS_BYTES = 128 * 128 * 2;     // one 128 x 128 fp16 operand (128B swizzle)
+  static constexpr int DS_BUFS = 1;                   // dS^T buffers (two measured slower at D = 64)
+  static constexpr int ROW_OFF = DS_OFF + DS_BUFS * DS_BYTES;   // stage s: lse2[128], delta[128]
   // dQ staging: per read-out warp two 4 KB boxes (32 rows x 32 fp32, 128-byte swizzle)
   static constexpr int DQS_OFF = ROW_OFF + NQ * 1024;
   static constexpr int BAR_OFF = DQS_OFF + 4 * 8192;
-  static constexpr int NBARS = 1 + 2 * NQ + 5 + 4 + 2;
+  static constexpr int NBARS = 1 + 2 * NQ + 6 + 4 + 2 + 1;
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
@@ -64,7 +87,8 @@ struct BwdCfg {
 
 struct BwdParams {
   const float* lse2;     // [B*Hq, Lq_pad]  LSE * log2(e), +inf on rows without keys / padding
-  const float* delta;    // [B*Hq, Lq_pad]
+  const float* delta;    // [B*Hq, Lq_pad]  Delta times the dO and V scales
+  const uint32_t* amax;  // largest |q|, |k|, |v|, |dO| (float bits)
   void* dk;              // [B, Lk, Hkv, D]
   void* dv;
   int B, Hq, Hkv, Lq, Lk, Lq_pad;
@@ -87,40 +111,121 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
-// Delta = rowsum(dO * O) and the log2-scaled LSE, both padded to Lq_pad rows.
-// Thread per (b, i, h) row with h fastest, so a warp reads neighbouring rows.
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* o, const uint16_t* dO, const float* lse,
-                                                      float* lse2, float* delta, int B, int Hq, int Lq,
-                                                      int Lq_pad, int D) {
-  const size_t n = size_t(B) * Lq_pad * Hq;
-  for (size_t t = blockIdx.x * size_t(blockDim.x) + threadIdx.x; t < n; t += size_t(gridDim.x) * blockDim.x) {
-    const int h = static_cast<int>(t % Hq);
-    const size_t bi = t / Hq;
-    const int i = static_cast<int>(bi % Lq_pad);
-    const int b = static_cast<int>(bi / Lq_pad);
-    const size_t dst = (size_t(b) * Hq + h) * Lq_pad + i;
-    if (i >= Lq) { lse2[dst] = INFINITY; delta[dst] = 0.f; continue; }
-    const size_t row = ((size_t(b) * Lq + i) * Hq + h) * D;
-    const uint4* po = reinterpret_cast<const uint4*>(o + row);
-    const uint4* pd = reinterpret_cast<const uint4*>(dO + row);
-    float acc = 0.f;
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 a = po[c], g = pd[c];
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
+// Power-of-two input scales.  k maps the largest magnitude into [2^t, 2^(t+1))
+// (0 for an all-zero, subnormal-only, inf or NaN tensor), clamped to [-60, 60]
+// so that every factor and its products stay finite in fp32.
+__device__ __forceinline__ int bwd_pow2_exp(uint32_t amax_bits, int t) {
+  const int e = static_cast<int>((amax_bits >> 23) & 0xffu);
+  if (e == 0 || e == 255) return 0;
+  return max(-60, min(60, t - (e - 127)));
+}
+__device__ __forceinline__ float bwd_pow2(int k) { return __int_as_float((127 + k) << 23); }
+struct BwdScales {
+  int kq, kk, kv, kdo;
+};
+// Q, K, V to [2^7, 2^8); dO to [2^(5-log2 D), 2^(6-log2 D)), so that
+// |dP^T|, |Delta| <= D * |dO| * |V| < 2^14 and |dS^T| < 2^15 (fp16: 65504).
+__device__ __forceinline__ BwdScales bwd_scales(const uint32_t* amax, int D) {
+  BwdScales sc;
+  sc.kq = bwd_pow2_exp(amax[0], 7);
+  sc.kk = bwd_pow2_exp(amax[1], 7);
+  sc.kv = bwd_pow2_exp(amax[2], 7);
+  sc.kdo = bwd_pow2_exp(amax[3], D == 128 ? -2 : -1);
+  return sc;
+}
+
+// Largest |x| of q, k, v, dO (bf16) into amax[0..3] (float bits; zeroed
+// before).  blockIdx.y picks the tensor; one atomic per block.
+__global__ void __launch_bounds__(256) bwd_amax_kernel(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                                       const uint16_t* dO, size_t nq, size_t nk, uint32_t* amax) {
+  __shared__ uint32_t wmax[8];
+  const int t = static_cast<int>(blockIdx.y);
+  const uint16_t* src = t == 0 ? q : t == 1 ? k : t == 2 ? v : dO;
+  const uint4* p4 = reinterpret_cast<const uint4*>(src);
+  const size_t n8 = ((t == 1 || t == 2) ? nk : nq) / 8;   // element counts are multiples of D (64 or 128)
+  const size_t stride = size_t(gridDim.x) * blockDim.x;
+  uint32_t m = 0;
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n8; i += 4 * stride) {
+    uint4 w[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
-        acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(gv[e] & 0xffff0000u), acc);
-      }
+    for (int u = 0; u < 4; ++u) w[u] = (i + u * stride < n8) ? p4[i + u * stride] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m = max(m, max(ws[e] & 0x7fffu, (ws[e] >> 16) & 0x7fffu));
     }
-    const float l = lse[(size_t(b) * Hq + h) * Lq + i];
-    lse2[dst] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-    delta[dst] = acc;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) m = max(m, wmax[w]);
+    if (m != 0) atomicMax(&amax[t], m << 16);      // |x| as float bits
   }
 }
 
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float* acc, void* dq, size_t n, float scale,
-                                                       int g_fp32) {
+// Delta = rowsum(dO * O) and the log2-scaled LSE, both padded to Lq_pad rows;
+// also the scaled fp16 copies of q and dO.  Delta carries the dO and V scales
+// of the dP^T products.  One thread per 8-element chunk of a (b, i, h) row,
+// h fastest, so that a warp reads and writes contiguous memory; the D / 8
+// threads of a row sum Delta with shuffles.
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* o, const uint16_t* dO, const uint16_t* q,
+                                                      const float* lse, const uint32_t* amax, float* lse2,
+                                                      float* delta, uint16_t* q16, uint16_t* do16, int B, int Hq,
+                                                      int Lq, int Lq_pad, int D) {
+  const BwdScales sc = bwd_scales(amax, D);
+  const float fq = bwd_pow2(sc.kq), fdo = bwd_pow2(sc.kdo), fdelta = bwd_pow2(sc.kdo + sc.kv);
+  const int cpr = D / 8;                           // chunks per row: 8 or 16, a power of two dividing 32
+  const size_t n = size_t(B) * Lq_pad * Hq * cpr;  // a multiple of 32: Lq_pad is a multiple of 128
+  for (size_t t = blockIdx.x * size_t(blockDim.x) + threadIdx.x; t < n; t += size_t(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(t % cpr);
+    const size_t rr = t / cpr;
+    const int h = static_cast<int>(rr % Hq);
+    const size_t bi = rr / Hq;
+    const int i = static_cast<int>(bi % Lq_pad);
+    const int b = static_cast<int>(bi / Lq_pad);
+    float acc = 0.f;
+    if (i < Lq) {
+      const size_t off = ((size_t(b) * Lq + i) * Hq + h) * D / 8 + c;     // in 16-byte chunks
+      const uint4 a = reinterpret_cast<const uint4*>(o)[off];
+      const uint4 g = reinterpret_cast<const uint4*>(dO)[off];
+      const uint4 x = reinterpret_cast<const uint4*>(q)[off];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w}, xv[4] = {x.x, x.y, x.z, x.w};
+      uint32_t hq[4], hd[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float g0 = __uint_as_float(gv[e] << 16), g1 = __uint_as_float(gv[e] & 0xffff0000u);
+        acc = fmaf(__uint_as_float(av[e] << 16), g0, acc);
+        acc = fmaf(__uint_as_float(av[e] & 0xffff0000u), g1, acc);
+        hd[e] = pack_f16x2(g0 * fdo, g1 * fdo);
+        hq[e] = pack_f16x2(__uint_as_float(xv[e] << 16) * fq, __uint_as_float(xv[e] & 0xffff0000u) * fq);
+      }
+      reinterpret_cast<uint4*>(q16)[off] = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+      reinterpret_cast<uint4*>(do16)[off] = make_uint4(hd[0], hd[1], hd[2], hd[3]);
+    }
+    // the row's chunks are cpr consecutive lanes of one warp (every lane of the
+    // warp takes part: the loop bound is a multiple of 32)
+    for (int m = 1; m < cpr; m <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (c == 0) {
+      const size_t dst = (size_t(b) * Hq + h) * Lq_pad + i;
+      if (i >= Lq) {
+        lse2[dst] = INFINITY;
+        delta[dst] = 0.f;
+      } else {
+        const float l = lse[(size_t(b) * Hq + h) * Lq + i];
+        lse2[dst] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+        delta[dst] = acc * fdelta;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* acc, void* dq, size_t n, float scale_in,
+                                                       const uint32_t* amax, int D, int g_fp32) {
+  const BwdScales sc = bwd_scales(amax, D);
+  const float scale = scale_in * bwd_pow2(-(sc.kdo + sc.kv + sc.kk));   // dS^T carries dO, V scales; K its own
   for (size_t t = blockIdx.x * size_t(blockDim.x) + threadIdx.x; t < n / 4; t += size_t(gridDim.x) * blockDim.x) {
     const float4 v = reinterpret_cast<const float4*>(acc)[t];
     if (g_fp32) {
@@ -151,11 +256,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* dp_full = s_full + 1;                 // dP^T of the pair is in TMEM
   uint64_t* p_ready = dp_full + 1;
   uint64_t* ds_ready = p_ready + 1;
-  uint64_t* ds_free = ds_ready + 1;
-  uint64_t* dq_full = ds_free + 1;       // [2]
+  uint64_t* ds_free = ds_ready + 1;      // [2] per dS^T buffer
+  uint64_t* dq_full = ds_free + 2;       // [2]
   uint64_t* dq_free = dq_full + 2;       // [2]
   uint64_t* dkv_done = dq_free + 2;
   uint64_t* mma_done = dkv_done + 1;
+  uint64_t* kv_conv = mma_done + 1;               // K and V converted to fp16 in shared memory
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,10 +291,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(dp_full, 1);
     mbar_init(p_ready, 256);
     mbar_init(ds_ready, 256);
-    mbar_init(ds_free, 1);
+    mbar_init(&ds_free[0], 1);
+    mbar_init(&ds_free[1], 1);
     for (int u = 0; u < 2; ++u) { mbar_init(&dq_full[u], 1); mbar_init(&dq_free[u], 128); }
     mbar_init(dkv_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(kv_conv, 256);
     fence_mbar_init();
   }
   if (warp == 14) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
@@ -231,15 +339,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else if (warp == 13) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0 && npairs > 0) {
-      constexpr uint32_t ID_SS = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t ID_DVK = idesc_bf16_f32(128, D, false, true);     // dV, dK: B = dO / Q (MN-major)
-      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, true, true);       // dQ: A = dS (MN-major), B = K (MN-major)
+      constexpr uint32_t ID_SS = idesc_f16_f32(128, 128, false, false);    // S^T, dP^T
+      constexpr uint32_t ID_DVK = idesc_f16_f32(128, D, false, true);      // dV, dK: B = dO / Q (MN-major)
+      constexpr uint32_t ID_DQ = idesc_f16_f32(128, D, true, true);        // dQ: A = dS (MN-major), B = K (MN-major)
       const uint32_t k_base = smem_u32(smem + C::K_OFF), v_base = smem_u32(smem + C::V_OFF);
       const uint32_t q_base = smem_u32(smem + C::Q_OFF), ds_base = smem_u32(smem + C::DS_OFF);
-      const uint32_t dslo_base = smem_u32(smem + C::DSLO_OFF);
-      // P^T of queries 16kk..16kk+15 in TMEM: P_hi in columns 16kk..16kk+7, P_lo
-      // in the next 8 (over the S^T columns of those queries)
-      auto p_col = [](int kk) { return C::T_S + kk * 16; };
+      // P^T of queries 16kk..16kk+15 in TMEM: 8 columns (fp16 pairs) at the start
+      // of the S^T columns of query half kk / 4 that the compute warp has read
+      auto p_col = [](int kk) { return C::T_S + (kk >> 2) * 64 + (kk & 3) * 8; };
       auto kmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024); };
       auto mnmaj = [](uint32_t base, int kk) { return sdesc_sw128(base + kk * 2048, 16384, 1024); };
       auto issue_s = [&](int n) {
@@ -254,21 +361,20 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < D / 16; ++kk) umma_ss(tmem + C::T_DP, kmaj(v_base, kk), kmaj(da, kk), ID_SS, kk > 0);
         umma_commit(dp_full);
       };
-      bool ok = mbar_wait(kv_full, 0, lim, W_BWD_KV) && mbar_wait(&q_full[0], 0, lim, W_BWD_QF);
+      bool ok = mbar_wait(kv_conv, 0, lim, W_BWD_KV) && mbar_wait(&q_full[0], 0, lim, W_BWD_QF);
       tc_fence_after();
       if (ok) { issue_s(0); issue_dp(0); }
       for (int n = 0; ok && n < npairs; ++n) {
         const int s = n % NQ, bq = n % NB;
         const uint32_t qa = q_base + s * 2 * C::TILE, da = qa + C::TILE;
         const bool more = n + 1 < npairs;
+        const int db = n % C::DS_BUFS;
+        const uint32_t dsa = ds_base + db * C::DS_BYTES;   // this pair's dS^T buffer
         if (!(ok = mbar_wait(p_ready, n & 1, lim, W_BWD_P))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // dV += P_hi^T dO  (K = 128 queries)
+        for (int kk = 0; kk < 8; ++kk)      // dV += P^T dO  (K = 128 queries)
           umma_ts(tmem + C::T_DV, tmem + p_col(kk), mnmaj(da, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // dV += P_lo^T dO
-          umma_ts(tmem + C::T_DV, tmem + p_col(kk) + 8, mnmaj(da, kk), ID_DVK, 1u);
         // the next pair's S^T goes over P^T as soon as the dV products are issued
         // (the pipe runs them in order; the compute warps keep P in registers),
         // when its Q has a stage of its own (with one stage, Q(n+1) replaces
@@ -282,20 +388,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         if (!C::DQ_IN_DP && more) issue_dp(n + 1);   // dP^T was read by the dS^T phase
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // dK += dS_hi^T Q  (K = 128 queries)
-          umma_ss(tmem + C::T_DK, kmaj(ds_base, kk), mnmaj(qa, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)      // dK += dS_lo^T Q
-          umma_ss(tmem + C::T_DK, kmaj(dslo_base, kk), mnmaj(qa, kk), ID_DVK, 1u);
+        for (int kk = 0; kk < 8; ++kk)      // dK += dS^T Q  (K = 128 queries)
+          umma_ss(tmem + C::T_DK, kmaj(dsa, kk), mnmaj(qa, kk), ID_DVK, (n > 0 || kk > 0) ? 1u : 0u);
         if (!C::DQ_IN_DP && n >= NB) {      // this dQ buffer must have been read out (pair n - NB)
           if (!(ok = mbar_wait(&dq_free[bq], ((n / NB) - 1) & 1, lim, W_BWD_DQF))) break;
           tc_fence_after();
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)      // dQ = dS K  (K = 128 keys)
-          umma_ss(tmem + C::T_DQ + bq * D, mnmaj(ds_base, kk), mnmaj(k_base, kk), ID_DQ, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + C::T_DQ + bq * D, mnmaj(dsa, kk), mnmaj(k_base, kk), ID_DQ, kk > 0 ? 1u : 0u);
         umma_commit(&dq_full[bq]);
-        umma_commit(ds_free);
+        umma_commit(&ds_free[db]);
         umma_commit(&q_empty[s]);
         if (C::DQ_IN_DP && more) {          // dP^T(n+1) overwrites dQ(n): wait for its read-out
           if (!(ok = mbar_wait(&dq_free[0], n & 1, lim, W_BWD_DQF))) break;
@@ -323,8 +426,33 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int r = wq * 32 + lane;
     const int key = j * 128 + r;
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
-    const float sl2 = p.scale_log2;
-    for (int n = 0; n < npairs; ++n) {
+    const BwdScales sc_in = bwd_scales(p.amax, D);
+    const float sl2 = p.scale_log2 * bwd_pow2(-(sc_in.kq + sc_in.kk));   // S^T carries the Q and K scales
+    // K and V (bf16) to scaled fp16 in place, once, before the first product
+    bool npairs_ok = true;
+    if (npairs > 0) {
+      if (!mbar_wait_warp(kv_full, 0, lim, W_BWD_KV)) {
+        npairs_ok = false;
+      } else {
+        const float fk = bwd_pow2(sc_in.kk), fv = bwd_pow2(sc_in.kv);
+        uint4* kv4 = reinterpret_cast<uint4*>(smem + C::K_OFF);      // K then V, contiguous
+        constexpr int N16 = 2 * C::TILE / 16;
+#pragma unroll 4
+        for (int c = threadIdx.x; c < N16; c += 256) {
+          const float f = (c < C::TILE / 16) ? fk : fv;
+          const uint4 w = kv4[c];
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          uint32_t hs[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            hs[e] = pack_f16x2(__uint_as_float(ws[e] << 16) * f, __uint_as_float(ws[e] & 0xffff0000u) * f);
+          kv4[c] = make_uint4(hs[0], hs[1], hs[2], hs[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(kv_conv);
+      }
+    }
+    for (int n = 0; npairs_ok && n < npairs; ++n) {
       const int s = n % NQ;
       const int i = i0 + n / G;
       const float* lse2 = reinterpret_cast<const float*>(smem + C::ROW_OFF + s * 1024);
@@ -337,8 +465,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool ok = true;
       // Phase 1: P^T = 2^(S^T * scale - LSE) (masked) for this warp's 64 query
       // columns, 16 at a time: kept in registers (fp32) for phase 2 and stored
-      // as P_hi + P_lo over the 16 S^T columns they come from, the A operand of
-      // the dV products; published at once.
+      // as fp16 over S^T columns already read (8 columns per 16 queries, at the
+      // start of this half's region), the A operand of the dV products;
+      // published at once.
       float pv[64];
 #pragma unroll
       for (int sc = 0; sc < 4; ++sc) {
@@ -348,7 +477,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // the mask only matters where some key row of the warp starts after c0
         // (the causal diagonal, keys past Lk); elsewhere every column is allowed
         const bool masked = __any_sync(0xffffffffu, cmin > c0);
-        uint32_t phi[8], plo[8];
+        uint32_t ph[8];
 #pragma unroll
         for (int t4 = 0; t4 < 4; ++t4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + 4 * t4);
@@ -366,20 +495,16 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             pv[sc * 16 + 2 * t] = p0;
             pv[sc * 16 + 2 * t + 1] = p1;
-            phi[t] = pack_bf16x2(p0, p1);
-            float r0, r1;
-            resid_bf16x2(phi[t], p0, p1, r0, r1);
-            plo[t] = pack_bf16x2(r0, r1);
+            ph[t] = pack_f16x2(p0, p1);
           }
         }
-        tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + c0, phi);
-        tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + c0 + 8, plo);
+        tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + hh * 64 + sc * 8, ph);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready);
       // Phase 2: dS^T = P^T * (dP^T - Delta) into swizzled shared memory as
-      // dS_hi + dS_lo, 16 query columns at a time.
+      // fp16, 16 query columns at a time.
       if (!mbar_wait_warp(dp_full, n & 1, lim, W_BWD_SDP)) break;
       tc_fence_after();
 #pragma unroll
@@ -387,31 +512,31 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int c0 = hh * 64 + sc * 16;
         uint32_t dp[16];
         tmem_ld_32x32b_x16(tmem + lane_bits + C::T_DP + c0, dp);
-        uint32_t dhi[8], dlo[8];
+        uint32_t dh[8];
 #pragma unroll
         for (int t4 = 0; t4 < 4; ++t4) {
           const float4 d4 = *reinterpret_cast<const float4*>(dlt + c0 + 4 * t4);
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = 2 * t4 + u;
-            float e0, e1, s0, s1, r0, r1;
+            float e0, e1, s0, s1;
             fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -(u ? d4.z : d4.x),
                   -(u ? d4.w : d4.y));
             ffma2(s0, s1, pv[sc * 16 + 2 * t], pv[sc * 16 + 2 * t + 1], e0, e1, 0.f, 0.f);
-            dhi[t] = pack_bf16x2(s0, s1);
-            resid_bf16x2(dhi[t], s0, s1, r0, r1);
-            dlo[t] = pack_bf16x2(r0, r1);
+            dh[t] = pack_f16x2(s0, s1);
           }
         }
-        // the shared-memory operands of pair n - 1 must have been consumed
-        if (sc == 0 && n > 0 && !(ok = mbar_wait_warp(ds_free, (n - 1) & 1, lim, W_BWD_DSF))) break;
+        // the dS^T buffer's previous pair (n - DS_BUFS) must have been consumed
+        if (sc == 0 && n >= C::DS_BUFS &&
+            !(ok = mbar_wait_warp(&ds_free[n % C::DS_BUFS], ((n / C::DS_BUFS) - 1) & 1, lim, W_BWD_DSF)))
+          break;
         // query columns c0..c0+15: two 16-byte chunks of the 128-byte row of block hh (128B swizzle)
         const int blk = hh * 16384 + rowoff;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const int o16 = blk + (((sc * 2 + t) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(smem + C::DS_OFF + o16) = make_uint4(dhi[4 * t], dhi[4 * t + 1], dhi[4 * t + 2], dhi[4 * t + 3]);
-          *reinterpret_cast<uint4*>(smem + C::DSLO_OFF + o16) = make_uint4(dlo[4 * t], dlo[4 * t + 1], dlo[4 * t + 2], dlo[4 * t + 3]);
+          *reinterpret_cast<uint4*>(smem + C::DS_OFF + (n % C::DS_BUFS) * C::DS_BYTES + o16) =
+              make_uint4(dh[4 * t], dh[4 * t + 1], dh[4 * t + 2], dh[4 * t + 3]);
         }
       }
       if (!ok) break;
@@ -467,9 +592,13 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (have) tc_fence_after();
     const int key = j * 128 + r;
     const size_t krow = ((size_t(b) * p.Lk + key) * p.Hkv + hkv) * D;
+    // the input scales come out here: dV carries dO's, dK^T = dS^T Q carries
+    // those of dO, V and Q
+    const BwdScales sc_out = bwd_scales(p.amax, D);
+    const float mul_dv = bwd_pow2(-sc_out.kdo), mul_dk = p.scale * bwd_pow2(-(sc_out.kdo + sc_out.kv + sc_out.kq));
 #pragma unroll
     for (int which = 0; which < 2; ++which) {       // 0: dV, 1: dK (scaled)
-      const float mul = which ? p.scale : 1.f;
+      const float mul = which ? mul_dk : mul_dv;
       void* out = which ? p.dk : p.dv;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {

@@ -110,9 +110,15 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float q_scale,
  * k and the saved lse instead of being stored.  Reads q, k, v, o, dO (bf16)
  * and lse (fp32, as written by fa_fwd); writes dq [B,Lq,Hq,D], dk and dv
  * [B,Lk,Hkv,D] in grad_dtype (FA_BF16 or FA_FP32).  dk/dv of a kv head are the
- * sums over its Hq/Hkv query heads.  workspace is caller-owned device memory
- * of at least fa_bwd_workspace_size() bytes (256-byte aligned); its contents
- * on entry do not matter.
+ * sums over its Hq/Hkv query heads.  The products run on fp16 operands: each
+ * input tensor is scaled by a power of two (chosen on the device from its
+ * largest magnitude) so that its bf16 values convert to fp16 exactly, P and
+ * dS enter the products as fp16, and the scales are taken out of the results
+ * exactly; an input holding inf or NaN gives non-finite gradients.  workspace
+ * is caller-owned device memory of at least fa_bwd_workspace_size() bytes
+ * (256-byte aligned: the fp32 dQ accumulator, the LSE and Delta rows, the
+ * scaled fp16 copies of q and dO, the input maxima); its contents on entry do
+ * not matter.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D);
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
