@@ -56,6 +56,40 @@ def test_bwd_matches_oracle(case):
         check_close(dq, rq, bf16_output=bf, what=f"dQ {gdt}")
 
 
+def test_bwd_power_of_two_input_scales():
+    """The products run on fp16 after each input tensor is scaled by a power of
+    two chosen from its largest magnitude.  Scaling the caller's q, k, v, dO by
+    powers of two (o follows exactly, the LSE is unchanged) must therefore give
+    the same fp16 operands and gradients scaled exactly: dV by dO's factor, dK
+    by the product of dO's, V's and Q's, dQ by that of dO's, V's and K's.  dK
+    and dV are bit-identical (fixed accumulation order); dQ is summed by
+    reductions in any order.  dO at 2^-20 of unit scale would be subnormal in
+    an unscaled fp16 copy."""
+    B, Hq, Hkv, Lq, Lk, D, causal = 1, 2, 1, 200, 200, 64, True
+    x = synth.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=11, with_do=True)
+    scale = 1.0 / math.sqrt(D)
+    eq, ek, ev, edo = -10, 10, 12, -20
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.fwd(q, k, v, scale=scale, causal=causal)
+    dq, dk, dv = fa.bwd(q, k, v, o, do, lse, scale=scale, causal=causal, grad_dtype=torch.float32)
+    qs, ks, vs, dos, os_ = q * 2.0 ** eq, k * 2.0 ** ek, v * 2.0 ** ev, do * 2.0 ** edo, o * 2.0 ** ev
+    for a, b_, e in ((qs, q, eq), (ks, k, ek), (vs, v, ev), (dos, do, edo), (os_, o, ev)):
+        assert a.dtype == torch.bfloat16 and torch.equal(a.float(), b_.float() * 2.0 ** e)   # exact in bf16
+    dq2, dk2, dv2 = fa.bwd(qs, ks, vs, os_, dos, lse, scale=scale, causal=causal, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(dv2, dv * 2.0 ** edo)
+    assert torch.equal(dk2, dk * 2.0 ** (edo + ev + eq))
+    torch.testing.assert_close(dq2, dq * 2.0 ** (edo + ev + ek), rtol=1e-5, atol=0.0)
+    # and against the oracle on the scaled inputs, errors measured at unit scale
+    xf = {n: synth.as_f64(x[n]) for n in x}
+    xf["q"] = xf["q"] * 2.0 ** eq; xf["k"] = xf["k"] * 2.0 ** ek
+    xf["v"] = xf["v"] * 2.0 ** ev; xf["do"] = xf["do"] * 2.0 ** edo
+    rq, rk, rv, *_ = oracle.attn_bwd(xf["q"], xf["k"], xf["v"], xf["do"], scale, causal)
+    check_close(f64(dv2) / 2.0 ** edo, rv / 2.0 ** edo, bf16_output=False, what="dV scaled inputs")
+    check_close(f64(dk2) / 2.0 ** (edo + ev + eq), rk / 2.0 ** (edo + ev + eq), bf16_output=False, what="dK scaled inputs")
+    check_close(f64(dq2) / 2.0 ** (edo + ev + ek), rq / 2.0 ** (edo + ev + ek), bf16_output=False, what="dQ scaled inputs")
+
+
 def test_bwd_empty_queries():
     k = torch.randn(1, 64, 2, 64, device="cuda").to(torch.bfloat16)
     q = torch.empty(1, 0, 2, 64, device="cuda", dtype=torch.bfloat16)
