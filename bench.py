@@ -435,20 +435,51 @@ def run_ours(args):
     value = whole_job_tflops(flops, world, args.steps, kernel_ms)
     tf_rank = flops / (ms_step * 1e-3) / 1e12
 
-    # end to end through the public API: pinned host inputs -> device -> fwd -> host
+    # end to end through the public API: every step copies its inputs from
+    # pinned host memory to the device, runs the forward and reads O and the LSE
+    # back.  Steps are pipelined over two buffer sets: step i's inputs go in on
+    # one copy stream while step i - 1's result comes back on another (PCIe is
+    # full duplex) and the forward runs on a third.
     hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
-    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
+    hl = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+    din = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)) for _ in range(2)]
+    dout = [(torch.empty_like(o), torch.empty_like(lse)) for _ in range(2)]
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        fa.fwd(dq, dk, dv, scale=w.scale, causal=w.causal, out=o, lse=lse)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
-    e2e_ms = statistics.mean(time_steps(e2e_step, max(3, args.steps // 4), 3, flush, stream))
+    def e2e_run(n):
+        ran, back = [None, None], [None, None]     # per buffer set: its forward done / its result read back
+        t0 = torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if ran[b] is not None:
+                    s_in.wait_event(ran[b])           # the inputs of step i - 2 are no longer read
+                for d, h in zip(din[b], (hq, hk, hv)):
+                    d.copy_(h, non_blocking=True)
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(e_in)
+                if back[b] is not None:
+                    s_run.wait_event(back[b])         # the result of step i - 2 has been read back
+                fa.fwd(*din[b], scale=w.scale, causal=w.causal, out=dout[b][0], lse=dout[b][1])
+                ran[b] = torch.cuda.Event()
+                ran[b].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ran[b])
+                ho[b].copy_(dout[b][0], non_blocking=True)
+                hl[b].copy_(dout[b][1], non_blocking=True)
+                back[b] = torch.cuda.Event()
+                back[b].record(s_out)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+    e2e_run(3)
+    n_e2e = max(3, args.steps // 4)
+    e2e_ms = max_over_ranks(e2e_run(n_e2e), dist, dev) / n_e2e
 
     # kernel-only cross-check: the same call captured once in a CUDA graph and
     # replayed (no host work between the events but the replay itself)
@@ -463,7 +494,7 @@ def run_ours(args):
     except Exception as e:  # reported, never fatal: the headline does not depend on it
         graph_ms = str(e)[:200]
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    d2h = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
     e2e_val = flops * world / (e2e_ms * 1e-3) / 1e12
 
     sections = {}
@@ -505,7 +536,9 @@ def run_ours(args):
         "graph_replay_ms": (statistics.mean(graph_ms) if isinstance(graph_ms, list) else graph_ms),
         "roofline": roofline("tensor", tf_rank, peaks, peak_src, "TFLOP/s",
                              traffic=profiled_traffic("fwd_kernel causal_prefill"), algorithmic_bytes=fwd_bytes(w)),
-        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "schedule": "pinned host buffers; consecutive steps' H2D, forward and D2H overlapped on three "
+                            "streams over two device buffer sets"},
         "gpu_launches": args.steps,
         "clocks": ck,
         "sections": sections,
