@@ -26,13 +26,13 @@
 //                   (NQ stages)
 //        warp 13    tcgen05: S^T = K Q^T and dP^T = V dO^T into TMEM,
 //                   dV += P^T dO, dK += dS^T Q, dQ = dS K
-//        P^T (fp16) goes to TMEM over the S^T columns it comes from, dS^T
-//        (fp16) to swizzled shared memory.
+//        P^T (fp16) goes to TMEM over S^T columns already read, dS^T (fp16)
+//        to swizzled shared memory.
 //        warps 0-7  one thread per key row; warps w and w + 4 share a TMEM lane
 //                   quadrant and take 64 of the 128 query columns each (no row
 //                   reduction is needed: P = 2^(s - LSE)); causal / ragged mask
 //                   on the tiles that need it; P^T is published first (the dV
-//                   products, then the next pair's S^T, run while dS^T is
+//                   product, then the next pair's S^T, run while dS^T is
 //                   formed from P kept in registers)
 //        warps 8-11 one thread per query row: dQ tile from TMEM (two buffers at
 //                   D = 64) into a swizzled shared-memory box per warp, added to
