@@ -90,6 +90,24 @@ def test_bwd_power_of_two_input_scales():
     check_close(f64(dq2) / 2.0 ** (edo + ev + ek), rq / 2.0 ** (edo + ev + ek), bf16_output=False, what="dQ scaled inputs")
 
 
+def test_bwd_zero_and_nan_gradients():
+    """Input scales come from each tensor's largest magnitude: an all-zero dO
+    (largest magnitude 0, no scaling) gives exactly zero gradients, and a NaN
+    in dO gives non-finite gradients of its head, with the call itself fine."""
+    B, Hq, Hkv, Lq, Lk, D = 1, 2, 1, 130, 130, 64
+    x = synth.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=5, with_do=True)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = fa.fwd(q, k, v, causal=True)
+    dq, dk, dv = fa.bwd(q, k, v, o, torch.zeros_like(do), lse, causal=True, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dq) == 0 and torch.count_nonzero(dk) == 0 and torch.count_nonzero(dv) == 0
+    bad = do.clone()
+    bad[0, 7, 1, 3] = float("nan")
+    dq, dk, dv = fa.bwd(q, k, v, o, bad, lse, causal=True, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert not torch.isfinite(dv).all() and not torch.isfinite(dq).all()
+
+
 def test_bwd_empty_queries():
     k = torch.randn(1, 64, 2, 64, device="cuda").to(torch.bfloat16)
     q = torch.empty(1, 0, 2, 64, device="cuda", dtype=torch.bfloat16)
