@@ -528,7 +528,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   uint16_t* q16 = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(delta) + row_bytes);
   uint16_t* do16 = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(q16) + h_bytes);
   uint32_t* amax = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(do16) + h_bytes);
-  if (cudaMemsetAsync(dq_acc, 0, acc_bytes, st) != cudaSuccess || cudaMemsetAsync(amax, 0, 16, st) != cudaSuccess)
+  int* counter = reinterpret_cast<int*>(amax + 4);                 // the main kernel's work counter
+  if (cudaMemsetAsync(dq_acc, 0, acc_bytes, st) != cudaSuccess || cudaMemsetAsync(amax, 0, 32, st) != cudaSuccess)
     return FA_ERR_CUDA;
   {
     const size_t nq = size_t(B) * Lq * Hq * D, nk = size_t(B) * Lk * Hkv * D;
@@ -559,7 +560,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.Lq_pad = lq_pad;
   p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f; p.g_fp32 = (grad_dtype == FA_FP32);
   p.wait_limit_ns = g_wait_limit_ns.load();
-  const unsigned grid = static_cast<unsigned>(((Lk + 127) / 128) * B * Hkv);
+  // persistent: at most one CTA per SM, taking key tiles from the counter
+  p.num_items = static_cast<int>(((Lk + 127) / 128) * B * Hkv);
+  p.work_counter = counter;
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(std::min(p.num_items, sms));
   fa_status s;
   if (D == 128) s = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, mdq, p, grid, st) : launch_bwd<128, false>(mq, mk, mv, mdo, mdq, p, grid, st);
   else s = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, mdq, p, grid, st) : launch_bwd<64, false>(mq, mk, mv, mdo, mdq, p, grid, st);
