@@ -58,7 +58,7 @@ PROFILED_TRAFFIC = {
     "fwd_kernel<fp8> causal_prefill": {"sources": ("csrc/fa_fwd.cuh", "csrc/sm100.cuh"),
                                        "sha256_16": "644cd20e74d80560", "bytes": 50400256 + 3337728},
     "bwd_main_kernel train_fwd_bwd": {"sources": ("csrc/fa_bwd.cuh", "csrc/sm100.cuh"),
-                                      "sha256_16": "3018772f75206d8b", "bytes": 406921728 + 223515392},
+                                      "sha256_16": "2ce9742435305e4b", "bytes": 406921728 + 223515392},
     # captured on the first 16 sequences of the decode workload (1.35888 GB of KV
     # rows), scaled to a launch by the KV bytes it reads
     "decode_split_kernel splitkv_decode": {"sources": ("csrc/fa_decode.cuh", "csrc/sm100.cuh"),

@@ -535,98 +535,98 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_proxy_async_smem();
         mbar_arrive(&kv_conv[u]);
       }
-    for (int n = 0; npairs_ok && n < I.npairs; ++n) {
-      const int g = gp + n, s = g % NQ;
-      const int i = I.i0 + n / G;
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::ROW_OFF + s * 1024);
-      const float* dlt = lse2 + 128;
-      if (!(npairs_ok = mbar_wait_warp(s_full, g & 1, lim, W_BWD_SDP))) break;
-      tc_fence_after();
-      // allowed when key <= query + off, i.e. column c >= cmin (nothing for keys past Lk)
-      const int cmin = key < p.Lk ? (CAUSAL ? key - off - i * 128 : -1) : (1 << 30);
-      const int rowoff = r * 128;
-      bool ok = true;
-      // Phase 1: P^T = 2^(S^T * scale - LSE) (masked) for this warp's 64 query
-      // columns, 16 at a time: kept in registers (fp32) for phase 2 and stored
-      // as fp16 over S^T columns already read (8 columns per 16 queries, at the
-      // start of this half's region), the A operand of the dV products;
-      // published at once.
-      float pv[64];
+      for (int n = 0; npairs_ok && n < I.npairs; ++n) {
+        const int g = gp + n, s = g % NQ;
+        const int i = I.i0 + n / G;
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::ROW_OFF + s * 1024);
+        const float* dlt = lse2 + 128;
+        if (!(npairs_ok = mbar_wait_warp(s_full, g & 1, lim, W_BWD_SDP))) break;
+        tc_fence_after();
+        // allowed when key <= query + off, i.e. column c >= cmin (nothing for keys past Lk)
+        const int cmin = key < p.Lk ? (CAUSAL ? key - off - i * 128 : -1) : (1 << 30);
+        const int rowoff = r * 128;
+        bool ok = true;
+        // Phase 1: P^T = 2^(S^T * scale - LSE) (masked) for this warp's 64 query
+        // columns, 16 at a time: kept in registers (fp32) for phase 2 and stored
+        // as fp16 over S^T columns already read (8 columns per 16 queries, at the
+        // start of this half's region), the A operand of the dV products;
+        // published at once.
+        float pv[64];
 #pragma unroll
-      for (int sc = 0; sc < 4; ++sc) {
-        const int c0 = hh * 64 + sc * 16;              // first query column of this sub-chunk
-        uint32_t sv[16];
-        tmem_ld_32x32b_x16(tmem + lane_bits + C::T_S + c0, sv);
-        // the mask only matters where some key row of the warp starts after c0
-        // (the causal diagonal, keys past Lk); elsewhere every column is allowed
-        const bool masked = __any_sync(0xffffffffu, cmin > c0);
-        uint32_t ph[8];
+        for (int sc = 0; sc < 4; ++sc) {
+          const int c0 = hh * 64 + sc * 16;              // first query column of this sub-chunk
+          uint32_t sv[16];
+          tmem_ld_32x32b_x16(tmem + lane_bits + C::T_S + c0, sv);
+          // the mask only matters where some key row of the warp starts after c0
+          // (the causal diagonal, keys past Lk); elsewhere every column is allowed
+          const bool masked = __any_sync(0xffffffffu, cmin > c0);
+          uint32_t ph[8];
 #pragma unroll
-        for (int t4 = 0; t4 < 4; ++t4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + 4 * t4);
+          for (int t4 = 0; t4 < 4; ++t4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + 4 * t4);
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int t = 2 * t4 + u;
-            const int c = c0 + 2 * t;
-            float x0, x1;
-            ffma2(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), sl2, sl2,
-                  -(u ? l4.z : l4.x), -(u ? l4.w : l4.y));
-            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            if (masked) {
-              p0 = (c >= cmin) ? p0 : 0.f;
-              p1 = (c + 1 >= cmin) ? p1 : 0.f;
+            for (int u = 0; u < 2; ++u) {
+              const int t = 2 * t4 + u;
+              const int c = c0 + 2 * t;
+              float x0, x1;
+              ffma2(x0, x1, __uint_as_float(sv[2 * t]), __uint_as_float(sv[2 * t + 1]), sl2, sl2,
+                    -(u ? l4.z : l4.x), -(u ? l4.w : l4.y));
+              float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              if (masked) {
+                p0 = (c >= cmin) ? p0 : 0.f;
+                p1 = (c + 1 >= cmin) ? p1 : 0.f;
+              }
+              pv[sc * 16 + 2 * t] = p0;
+              pv[sc * 16 + 2 * t + 1] = p1;
+              ph[t] = pack_f16x2(p0, p1);
             }
-            pv[sc * 16 + 2 * t] = p0;
-            pv[sc * 16 + 2 * t + 1] = p1;
-            ph[t] = pack_f16x2(p0, p1);
+          }
+          tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + hh * 64 + sc * 8, ph);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+        // Phase 2: dS^T = P^T * (dP^T - Delta) into swizzled shared memory as
+        // fp16, 16 query columns at a time.
+        if (!(npairs_ok = mbar_wait_warp(dp_full, g & 1, lim, W_BWD_SDP))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int sc = 0; sc < 4; ++sc) {
+          const int c0 = hh * 64 + sc * 16;
+          uint32_t dp[16];
+          tmem_ld_32x32b_x16(tmem + lane_bits + C::T_DP + c0, dp);
+          uint32_t dh[8];
+#pragma unroll
+          for (int t4 = 0; t4 < 4; ++t4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dlt + c0 + 4 * t4);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int t = 2 * t4 + u;
+              float e0, e1, s0, s1;
+              fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -(u ? d4.z : d4.x),
+                    -(u ? d4.w : d4.y));
+              ffma2(s0, s1, pv[sc * 16 + 2 * t], pv[sc * 16 + 2 * t + 1], e0, e1, 0.f, 0.f);
+              dh[t] = pack_f16x2(s0, s1);
+            }
+          }
+          // the dS^T buffer's previous pair (g - DS_BUFS) must have been consumed
+          if (sc == 0 && g >= C::DS_BUFS &&
+              !(ok = mbar_wait_warp(&ds_free[g % C::DS_BUFS], ((g / C::DS_BUFS) - 1) & 1, lim, W_BWD_DSF)))
+            break;
+          // query columns c0..c0+15: two 16-byte chunks of the 128-byte row of block hh (128B swizzle)
+          const int blk = hh * 16384 + rowoff;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int o16 = blk + (((sc * 2 + t) ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(smem + C::DS_OFF + (g % C::DS_BUFS) * C::DS_BYTES + o16) =
+                make_uint4(dh[4 * t], dh[4 * t + 1], dh[4 * t + 2], dh[4 * t + 3]);
           }
         }
-        tmem_st_32x32b_x8(tmem + lane_bits + C::T_S + hh * 64 + sc * 8, ph);
+        if (!(npairs_ok = ok)) break;
+        fence_proxy_async_smem();
+        tc_fence_before();                               // the phase-2 reads of dP^T come first
+        mbar_arrive(ds_ready);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_ready);
-      // Phase 2: dS^T = P^T * (dP^T - Delta) into swizzled shared memory as
-      // fp16, 16 query columns at a time.
-      if (!(npairs_ok = mbar_wait_warp(dp_full, g & 1, lim, W_BWD_SDP))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int sc = 0; sc < 4; ++sc) {
-        const int c0 = hh * 64 + sc * 16;
-        uint32_t dp[16];
-        tmem_ld_32x32b_x16(tmem + lane_bits + C::T_DP + c0, dp);
-        uint32_t dh[8];
-#pragma unroll
-        for (int t4 = 0; t4 < 4; ++t4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(dlt + c0 + 4 * t4);
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int t = 2 * t4 + u;
-            float e0, e1, s0, s1;
-            fadd2(e0, e1, __uint_as_float(dp[2 * t]), __uint_as_float(dp[2 * t + 1]), -(u ? d4.z : d4.x),
-                  -(u ? d4.w : d4.y));
-            ffma2(s0, s1, pv[sc * 16 + 2 * t], pv[sc * 16 + 2 * t + 1], e0, e1, 0.f, 0.f);
-            dh[t] = pack_f16x2(s0, s1);
-          }
-        }
-        // the dS^T buffer's previous pair (g - DS_BUFS) must have been consumed
-        if (sc == 0 && g >= C::DS_BUFS &&
-            !(ok = mbar_wait_warp(&ds_free[g % C::DS_BUFS], ((g / C::DS_BUFS) - 1) & 1, lim, W_BWD_DSF)))
-          break;
-        // query columns c0..c0+15: two 16-byte chunks of the 128-byte row of block hh (128B swizzle)
-        const int blk = hh * 16384 + rowoff;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int o16 = blk + (((sc * 2 + t) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(smem + C::DS_OFF + (g % C::DS_BUFS) * C::DS_BYTES + o16) =
-              make_uint4(dh[4 * t], dh[4 * t + 1], dh[4 * t + 2], dh[4 * t + 3]);
-        }
-      }
-      if (!(npairs_ok = ok)) break;
-      fence_proxy_async_smem();
-      tc_fence_before();                               // the phase-2 reads of dP^T come first
-      mbar_arrive(ds_ready);
-    }
       ++it;
       gp += I.npairs;
     }
