@@ -117,8 +117,9 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float q_scale,
  * exactly; an input holding inf or NaN gives non-finite gradients.  workspace
  * is caller-owned device memory of at least fa_bwd_workspace_size() bytes
  * (256-byte aligned: the fp32 dQ accumulator, the LSE and Delta rows, the
- * scaled fp16 copies of q and dO, the input maxima); its contents on entry do
- * not matter.
+ * scaled fp16 copies of q and dO, the input maxima and the main kernel's work
+ * counter); its contents on entry do not matter.  Calls that share one
+ * workspace must be ordered on one stream.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Lq, int D);
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
